@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the verifier hot path: verified tokens/s of one decode verify
+step at concurrency 32 — 32 sequences x (K+1 = 4) rows = 128 tokens through 12
+MoE feed-forward layers (64 routed + 2 shared SwiGLU experts, top-6, hidden
+1280, width 896), then the LM-head argmax over 129,280 tokens and the
+longest-prefix accept with the bonus token.
+
+One rank per GPU (torchrun for N > 1); every rank verifies its own batch of 32
+sequences with its own copy of the weights (data-parallel replicas, weak
+scaling, no collective on the data path). Rank 0 prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl vgv|reference]
+
+Inputs are seeded synthetic tensors drawn on the device (weights N(0, 0.02),
+hidden states N(0, 1), bf16). Drafts follow the draft model of the workload:
+each drafted token equals the verifier's argmax with probability 0.576, else a
+uniform token; the argmax is taken from an untimed pass of the same step.
+The 5.78 GB of weights streamed per step exceed the 126 MB L2, so no flush is
+needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+B, K, T, LAYERS = 32, 3, 128, 12
+H, I, E, S, TOPK, V = 1280, 896, 64, 2, 6, 129280
+P_DRAFT = 0.576
+SEED = 0
+CFG = 1
+METRIC = "verified tokens/s, MoE verify step B=32 K=3"
+UNIT = "tokens/s"
+WORKLOAD = {
+    "workload": "decode verify step: B=32 seqs x (K+1)=4 rows = 128 tokens, 12 MoE FFN layers "
+                "(64 routed + 2 shared SwiGLU experts, top-6, H=1280, I=896) + LM-head argmax over "
+                "129,280 + prefix accept",
+    "B": B, "K": K, "tokens": T, "layers": LAYERS, "vocab": V, "draft_p": P_DRAFT,
+    "l2": "inputs larger than L2: 5.78 GB of weights per step vs 126 MB L2, no flush",
+}
+GATE_UP_W_BYTES = 2 * I * H * 2  # gate + up rows of one expert, bf16
+
+
+def _env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ oracle leg
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_step_sample(seed: int = SEED, n_sample: int = 2):
+    """Times the CPU oracle on a bounded sample of the step and scales it to a
+    whole step. Sample: n_sample of the 12 MoE layers over all 128 tokens (the
+    time of a layer is counted 12/n_sample times) plus the full LM-head argmax
+    and accept over the 128 rows. Inputs come from the numpy generator (same
+    distributions as the GPU leg) and are drawn once per process."""
+    import numpy as np
+
+    import oracle
+    import synth_inputs as si
+
+    d = si.FULL
+    key = (seed, n_sample)
+    if key not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS[key] = ([si.layer_weights(seed, CFG, l, d) for l in range(n_sample)],
+                               si.lm_head(seed, CFG, V, H), si.hidden_states(seed, CFG, T, H))
+    layers, lm, x = _ORACLE_INPUTS[key]
+    t0 = time.perf_counter()
+    h, _ = oracle.moe_stack(x, layers, k=TOPK, I=I)
+    t_layers = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    arg, _ = oracle.lm_head_argmax(h, lm)
+    drafts = si.drafts_from_argmax(arg, B, K, P_DRAFT, V, seed, CFG)
+    acc, _ = oracle.prefix_accept(arg, drafts, B, K)
+    t_verify = time.perf_counter() - t1
+    step_s = t_layers * (LAYERS / n_sample) + t_verify
+    tokens = int(np.sum(acc + 1))
+    return step_s, tokens, (f"{n_sample} of {LAYERS} MoE layers over {T} tokens (time x{LAYERS / n_sample:g}) + "
+                            f"full LM-head argmax/accept over {T} rows")
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_step_sample()
+    times, toks, sample = [], 0, ""
+    for _ in range(args.steps):
+        s, toks, sample = oracle_step_sample()
+        times.append(s)
+    step_s = statistics.mean(times)
+    value = toks / step_s
+    cores = _cores()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": dict(WORKLOAD, parallelism="host cores"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def run_gpu(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import greedy_speculative_verify_b200 as vgv
+    import synth_inputs as si
+    from greedy_speculative_verify_b200 import build as vbuild
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0 and not vbuild.up_to_date():
+        vbuild.build()
+    if world > 1:
+        dist.barrier()
+    vgv.load()
+    d = si.FULL
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- inputs (weights identical on every rank, the batch differs per rank)
+    layers = [si.torch_layer_weights(SEED, CFG, l, d, device=dev) for l in range(LAYERS)]
+    rw = [l["router_w"] for l in layers]
+    ew = [l["expert_w"] for l in layers]
+    sw = [l["shared_w"] for l in layers]
+    lm = si.torch_normal_bf16((V, H), 0.02, SEED, CFG, si.TID_LM_HEAD, device=dev)
+    x = si.torch_normal_bf16((T, H), 1.0, SEED + 1000 * rank, CFG, si.TID_X, device=dev)
+    hid = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    drafts = torch.zeros(B, K, dtype=torch.int32, device=dev)
+    argmax = torch.empty(T, dtype=torch.int32, device=dev)
+    accepted = torch.empty(B, dtype=torch.int32, device=dev)
+    toks = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
+    ws_stack = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device=dev)
+    ws_ver = torch.empty(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
+
+    def step(x_in, d_in):
+        vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, T, x_in, rw, None, ew, sw, hid, ws_stack)
+        vgv.vg_verify_greedy(B, K, H, V, hid, lm, d_in, argmax, accepted, toks, ws_ver)
+
+    # ---- drafts: the verifier's own argmax with probability p, else uniform
+    step(x, drafts)
+    torch.cuda.synchronize()
+    g = torch.Generator(device=dev)
+    g.manual_seed(SEED + 17 + rank)
+    a = argmax.view(B, K + 1)[:, :K]
+    u = torch.rand(B, K, generator=g, device=dev)
+    noise = torch.randint(0, V, (B, K), generator=g, device=dev, dtype=torch.int32)
+    drafts.copy_(torch.where(u < P_DRAFT, a, noise))
+
+    # ---- gate/up launch bytes per layer, from each layer's routing (untimed)
+    n_touched = []
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    ws_one = torch.empty(vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device=dev)
+    cur, nxt = x.clone(), torch.empty_like(x)
+    for l in range(LAYERS):
+        vgv.vg_moe_ffn(vgv.MOE_DIMS, T, cur, rw[l], None, ew[l], sw[l], 1, nxt, vgv.make_taps(expert_offsets=off), ws_one)
+        n_touched.append(int((off[1:] - off[:-1] > 0).sum().item()))
+        cur, nxt = nxt, cur
+    del ws_one
+    N = T * TOPK
+    act_bytes = N * H * 2 + T * H * 2 + (N + S * T) * I * 2
+    gate_up_bytes = [(n + S) * GATE_UP_W_BYTES + act_bytes for n in n_touched]
+
+    # ---- device-timed region: the whole step replayed from a CUDA graph
+    step(x, drafts)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(x, drafts)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    # keep the GPU under load for about a second so the clock samples see it
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        graph.replay()
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    tokens_rank = int((accepted.to(torch.int64) + 1).sum().item())
+    st, info = vgv.vg_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {vgv.STATUS_NAMES.get(st, st)} at site {info}")
+
+    # ---- end to end through the public calls: pinned host inputs in, results out
+    x_host = x.cpu().pin_memory()
+    d_host = drafts.cpu().pin_memory()
+    acc_host = torch.empty(B, dtype=torch.int32).pin_memory()
+    tok_host = torch.empty(B, K + 1, dtype=torch.int32).pin_memory()
+    x_in = torch.empty_like(x)
+    d_in = torch.empty_like(drafts)
+
+    def e2e_step():
+        x_in.copy_(x_host, non_blocking=True)
+        d_in.copy_(d_host, non_blocking=True)
+        step(x_in, d_in)
+        acc_host.copy_(accepted, non_blocking=True)
+        tok_host.copy_(toks, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    ev1.synchronize()
+    barrier()
+    e2e_ms = ev0.elapsed_time(ev1) / args.steps
+    assert int((acc_host.to(torch.int64) + 1).sum()) == tokens_rank
+    h2d = x_host.numel() * x_host.element_size() + d_host.numel() * d_host.element_size()
+    d2h = acc_host.numel() * acc_host.element_size() + tok_host.numel() * tok_host.element_size()
+
+    # ---- kernel timing: CUDA events around every launch, on the launch stream
+    kr = max(1, min(args.steps, 10))
+    kinds = {vgv.VG_KERNEL_ROUTER: "router", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_GATE_UP: "gate_up",
+             vgv.VG_KERNEL_DOWN: "down", vgv.VG_KERNEL_COMBINE: "combine", vgv.VG_KERNEL_LM_HEAD: "lm_head",
+             vgv.VG_KERNEL_ACCEPT: "accept"}
+    per_step = {k: (1 if k in (vgv.VG_KERNEL_LM_HEAD, vgv.VG_KERNEL_ACCEPT) else LAYERS) for k in kinds}
+    evs = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)],
+               [torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)]) for k in kinds}
+    for k, (a0, a1) in evs.items():
+        vgv.vg_profile_set_events(k, a0, a1)
+    for _ in range(kr):
+        step(x, drafts)
+    torch.cuda.synchronize()
+    counts = {k: vgv.vg_profile_count(k) for k in kinds}
+    for k in kinds:
+        vgv.vg_profile_set_events(k, [], [])
+    dur = {k: [s.elapsed_time(e) for s, e in zip(*evs[k])] for k in kinds}
+    breakdown = {kinds[k]: sum(dur[k]) / kr for k in kinds}
+    gu = dur[vgv.VG_KERNEL_GATE_UP]
+    gu_bytes = sum(gate_up_bytes[i % LAYERS] for i in range(len(gu)))
+    achieved = gu_bytes / (sum(gu) / 1e3) / 1e9
+    launches_per_step = sum(counts.values()) // kr
+    grouping_kernels = 1 if T * TOPK <= 8192 else 3
+    launches_per_step += (grouping_kernels - 1) * LAYERS
+
+    # ---- aggregate over ranks (max time, summed tokens)
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+        n = torch.tensor([tokens_rank], dtype=torch.int64, device=dev)
+        dist.all_reduce(n)
+        tokens_all = int(n.item())
+    else:
+        tokens_all = tokens_rank
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s_step, s_tok, sample = oracle_step_sample()
+        cpu = {"value": s_tok / s_step, "unit": UNIT, "cores": _cores(), "kind": "oracle", "sample": sample}
+
+    peak, peak_kind = _peaks()
+    line = {
+        "metric": METRIC, "value": tokens_all / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism=f"replicas x{world}", cuda_graph=True),
+        "tokens_per_step": tokens_all, "tau": tokens_rank / B,
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "gate_up (grouped gate/up GEMM + SwiGLU)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
+                     "algorithmic_bytes_per_launch": gu_bytes / max(1, len(gu)),
+                     "avg_launch_ms": sum(gu) / max(1, len(gu))},
+        "breakdown_ms_per_step": breakdown,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["vgv", "reference"], default="vgv")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = _env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_gpu(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

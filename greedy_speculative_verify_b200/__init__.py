@@ -1,0 +1,195 @@
+"""Python binding of the verifier hot-path library (libvgv.so, include/vgv.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libvgv.so. The functions carry the C names and take torch tensors
+(device memory, any stream) or ``None``; they return nothing and raise
+``VgError`` on a non-OK status. There is no CPU fallback: if the library is not
+built, the first call raises.
+
+    import greedy_speculative_verify_b200 as vgv
+    ws = torch.empty(vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device="cuda")
+    vgv.vg_moe_ffn(vgv.MOE_DIMS, T, x, router_w, None, expert_w, shared_w, 1, out, None, ws)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvgv.so")
+
+VG_OK = 0
+STATUS_NAMES = {0: "VG_OK", 1: "VG_ERR_INVALID_ARG", 2: "VG_ERR_UNSUPPORTED", 3: "VG_ERR_WORKSPACE",
+                4: "VG_ERR_CUDA", 5: "VG_ERR_TIMEOUT", 6: "VG_ERR_DEVICE_BOUNDS"}
+
+# every symbol include/vgv.h declares
+EXPORTS = (
+    "vg_status_string", "vg_abi_version", "vg_moe_workspace_bytes", "vg_moe_ffn",
+    "vg_moe_stack_workspace_bytes", "vg_moe_ffn_stack", "vg_verify_workspace_bytes",
+    "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag",
+    "vg_profile_set_events", "vg_profile_count",
+)
+
+# vg_kernel
+VG_KERNEL_ROUTER, VG_KERNEL_GROUPING, VG_KERNEL_GATE_UP, VG_KERNEL_DOWN = 0, 1, 2, 3
+VG_KERNEL_COMBINE, VG_KERNEL_LM_HEAD, VG_KERNEL_ACCEPT = 4, 5, 6
+
+
+class VgError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class vg_moe_dims(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("intermediate", ctypes.c_int32), ("n_routed", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+
+class vg_moe_taps(ctypes.Structure):
+    _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_weight", ctypes.c_void_p),
+                ("expert_offsets", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("inv_perm", ctypes.c_void_p),
+                ("act", ctypes.c_void_p), ("expert_out", ctypes.c_void_p)]
+
+
+MOE_DIMS = vg_moe_dims(1280, 896, 64, 2, 6)
+
+_lib = None
+
+
+def load():
+    """Loads libvgv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with greedy_speculative_verify_b200.build.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t
+    dims_p = ctypes.POINTER(vg_moe_dims)
+    sig = {
+        "vg_status_string": (ctypes.c_char_p, [i32]),
+        "vg_abi_version": (i32, []),
+        "vg_moe_workspace_bytes": (sz, [dims_p, i32]),
+        "vg_moe_ffn": (i32, [dims_p, i32, vp, vp, vp, vp, vp, i32, vp, ctypes.POINTER(vg_moe_taps), vp, sz, vp]),
+        "vg_moe_stack_workspace_bytes": (sz, [dims_p, i32]),
+        "vg_moe_ffn_stack": (i32, [dims_p, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                   ctypes.POINTER(vp), vp, vp, sz, vp]),
+        "vg_verify_workspace_bytes": (sz, [i32, i32, i32, i32]),
+        "vg_verify_greedy": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "vg_get_device_status": (i32, [vp, ctypes.POINTER(i32)]),
+        "vg_set_wait_timeout_ns": (i32, [u64]),
+        "vg_debug_wait_flag": (i32, [vp, i32, u64, vp]),
+        "vg_profile_set_events": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
+        "vg_profile_count": (ctypes.c_int64, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != VG_OK:
+        raise VgError(st, where)
+
+
+def vg_abi_version() -> int:
+    return load().vg_abi_version()
+
+
+def vg_status_string(s: int) -> str:
+    return load().vg_status_string(s).decode()
+
+
+def vg_moe_workspace_bytes(dims: vg_moe_dims, T_max: int) -> int:
+    return load().vg_moe_workspace_bytes(ctypes.byref(dims), T_max)
+
+
+def vg_moe_stack_workspace_bytes(dims: vg_moe_dims, T_max: int) -> int:
+    return load().vg_moe_stack_workspace_bytes(ctypes.byref(dims), T_max)
+
+
+def vg_verify_workspace_bytes(B: int, K: int, H: int, V: int) -> int:
+    return load().vg_verify_workspace_bytes(B, K, H, V)
+
+
+def make_taps(topk_idx=None, topk_weight=None, expert_offsets=None, perm=None, inv_perm=None, act=None,
+              expert_out=None) -> vg_moe_taps:
+    return vg_moe_taps(*(None if t is None else t.data_ptr()
+                         for t in (topk_idx, topk_weight, expert_offsets, perm, inv_perm, act, expert_out)))
+
+
+def vg_moe_ffn(dims, T, x, router_w, router_bias, expert_w, shared_w, add_residual, out, taps, workspace,
+               stream=None):
+    st = load().vg_moe_ffn(ctypes.byref(dims), T, _ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(expert_w),
+                           _ptr(shared_w), int(add_residual), _ptr(out),
+                           None if taps is None else ctypes.byref(taps), _ptr(workspace),
+                           0 if workspace is None else workspace.numel() * workspace.element_size(),
+                           _stream(stream))
+    _check(st, "vg_moe_ffn")
+
+
+def vg_moe_ffn_stack(dims, n_layers, T, x, router_w, router_bias, expert_w, shared_w, out, workspace, stream=None):
+    """router_w, expert_w, shared_w: sequences of n_layers tensors; router_bias:
+    None or a sequence of tensors/None."""
+    arr = ctypes.c_void_p * n_layers
+    rw = arr(*(t.data_ptr() for t in router_w))
+    ew = arr(*(t.data_ptr() for t in expert_w))
+    sw = arr(*(t.data_ptr() for t in shared_w))
+    rb = None if router_bias is None else arr(*(None if t is None else t.data_ptr() for t in router_bias))
+    st = load().vg_moe_ffn_stack(ctypes.byref(dims), n_layers, T, _ptr(x), rw, rb, ew, sw, _ptr(out),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "vg_moe_ffn_stack")
+
+
+def vg_verify_greedy(B, K, H, V, h, lm_head, drafts, argmax, accepted, out_tokens, workspace, stream=None):
+    st = load().vg_verify_greedy(B, K, H, V, _ptr(h), _ptr(lm_head), _ptr(drafts), _ptr(argmax), _ptr(accepted),
+                                 _ptr(out_tokens), _ptr(workspace),
+                                 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(st, "vg_verify_greedy")
+
+
+def vg_get_device_status(stream=None) -> tuple[int, int]:
+    """(status code, site) of the first fault recorded on the current device; clears it."""
+    info = ctypes.c_int32(0)
+    st = load().vg_get_device_status(_stream(stream), ctypes.byref(info))
+    return st, info.value
+
+
+def vg_set_wait_timeout_ns(ns: int):
+    _check(load().vg_set_wait_timeout_ns(ns), "vg_set_wait_timeout_ns")
+
+
+def vg_debug_wait_flag(flag, expect: int, max_ns: int, stream=None):
+    _check(load().vg_debug_wait_flag(_ptr(flag), expect, max_ns, _stream(stream)), "vg_debug_wait_flag")
+
+
+def vg_profile_set_events(kind: int, starts, stops):
+    """starts/stops: sequences of torch.cuda.Event (enable_timing=True); empty clears."""
+    n = len(starts)
+    arr = ctypes.c_void_p * max(n, 1)
+    a = arr(*(e.cuda_event for e in starts))
+    b = arr(*(e.cuda_event for e in stops))
+    _check(load().vg_profile_set_events(kind, a, b, n), "vg_profile_set_events")
+
+
+def vg_profile_count(kind: int) -> int:
+    return load().vg_profile_count(kind)

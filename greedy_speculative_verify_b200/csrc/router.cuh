@@ -1,0 +1,195 @@
+// Router of the MoE layer: fp32 logits, top-k selection and softmax gates.
+//
+// Top-6 of 64 routed experts per token ("Jina AI's 3.4B OCR model targets faster
+// page parsing", "A compressed visual front end"; jina-ocr-v1 model card,
+// architecture paragraph). The pages give no formula. Reading used here:
+//  * l[t,e] = fp32 fused-multiply-add chain over h = 0..H-1 starting at +0,
+//    then + bias[e] in one fp32 addition. The order is part of the definition
+//    so that the selected experts are reproducible bit for bit; both kernels
+//    below keep each output's chain in one thread, in increasing h.
+//  * selection by (l descending, e ascending); softmax over all E logits,
+//    weights not renormalised over the selected experts.
+#pragma once
+#include "common.cuh"
+
+namespace vg {
+
+constexpr int kRouterE = 64;
+
+__device__ __forceinline__ void fma8(float& acc, uint4 a, uint4 b) {
+  acc = __fmaf_rn(bf16_lo(a.x), bf16_lo(b.x), acc);
+  acc = __fmaf_rn(bf16_hi(a.x), bf16_hi(b.x), acc);
+  acc = __fmaf_rn(bf16_lo(a.y), bf16_lo(b.y), acc);
+  acc = __fmaf_rn(bf16_hi(a.y), bf16_hi(b.y), acc);
+  acc = __fmaf_rn(bf16_lo(a.z), bf16_lo(b.z), acc);
+  acc = __fmaf_rn(bf16_hi(a.z), bf16_hi(b.z), acc);
+  acc = __fmaf_rn(bf16_lo(a.w), bf16_lo(b.w), acc);
+  acc = __fmaf_rn(bf16_hi(a.w), bf16_hi(b.w), acc);
+}
+
+// One warp selects the top-K of 64 logits of one token and writes the expert
+// ids (descending logit, lower id first among equal logits) and the softmax
+// probabilities over all 64 at those ids.
+template <int K>
+__device__ __forceinline__ void topk_softmax_warp(const float* l, int lane, int32_t* idx_out, float* w_out) {
+  const float v0 = l[lane], v1 = l[lane + 32];
+  bool u0 = false, u1 = false;
+  float sel_v[K];
+  int sel_i[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    float bv;
+    int bi;
+    if (!u0 && (u1 || v0 >= v1)) {
+      bv = v0;
+      bi = lane;
+    } else if (!u1) {
+      bv = v1;
+      bi = lane + 32;
+    } else {
+      bv = -INFINITY;
+      bi = 1 << 30;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    sel_v[j] = bv;
+    sel_i[j] = bi;
+    if (bi == lane) u0 = true;
+    if (bi == lane + 32) u1 = true;
+  }
+  const float m = sel_v[0];
+  float s = expf(v0 - m) + expf(v1 - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    if (lane == j) {
+      idx_out[j] = sel_i[j];
+      w_out[j] = expf(sel_v[j] - m) / s;
+    }
+  }
+}
+
+// Small token counts: one thread per (token, expert) output, 4 tokens x 64
+// experts per block; operands stream from L1/L2 with 16-byte loads.
+template <int K>
+__global__ void __launch_bounds__(256) router_topk_small(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ w,
+                                                         const float* __restrict__ bias, int T, int H,
+                                                         int32_t* __restrict__ idx_out,
+                                                         float* __restrict__ w_out) {
+  __shared__ float logit[4][kRouterE];
+  const int tl = threadIdx.x >> 6, e = threadIdx.x & 63;
+  const int t = blockIdx.x * 4 + tl;
+  float acc = 0.0f;
+  if (t < T) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    const uint4* wr = reinterpret_cast<const uint4*>(w + (size_t)e * H);
+    const int nc = H / 8;
+#pragma unroll 4
+    for (int c = 0; c < nc; ++c) fma8(acc, __ldg(xr + c), __ldg(wr + c));
+    if (bias != nullptr) acc = __fadd_rn(acc, bias[e]);
+  }
+  logit[tl][e] = acc;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 4) {
+    const int tt = blockIdx.x * 4 + warp;
+    if (tt < T) topk_softmax_warp<K>(logit[warp], lane, idx_out + (size_t)tt * K, w_out + (size_t)tt * K);
+  }
+}
+
+// Large token counts: a 128-token x 64-expert block tile, staged through shared
+// memory 32 k at a time; each thread owns 8 tokens x 4 experts and runs every
+// output's chain in increasing k.
+template <int K>
+__global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ w,
+                                                         const float* __restrict__ bias, int T, int H,
+                                                         int32_t* __restrict__ idx_out,
+                                                         float* __restrict__ w_out) {
+  constexpr int BT = 128, BK = 32, XS = BT + 4, WS = kRouterE + 4, LS = kRouterE + 1;
+  __shared__ __align__(16) float buf[BT * LS];  // k-loop: xs[BK][XS] | ws[BK][WS]; after: logits[BT][LS]
+  float* xs = buf;
+  float* ws = buf + BK * XS;
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+  const int t0 = blockIdx.x * BT;
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+
+  for (int k0 = 0; k0 < H; k0 += BK) {
+    // x tile: 128 tokens x 32 k = 512 uint4
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int q = tid + r * 256;
+      const int tok = q >> 2, kq = (q & 3) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t0 + tok < T) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tok) * H + k0 + kq));
+      xs[(kq + 0) * XS + tok] = bf16_lo(v.x);
+      xs[(kq + 1) * XS + tok] = bf16_hi(v.x);
+      xs[(kq + 2) * XS + tok] = bf16_lo(v.y);
+      xs[(kq + 3) * XS + tok] = bf16_hi(v.y);
+      xs[(kq + 4) * XS + tok] = bf16_lo(v.z);
+      xs[(kq + 5) * XS + tok] = bf16_hi(v.z);
+      xs[(kq + 6) * XS + tok] = bf16_lo(v.w);
+      xs[(kq + 7) * XS + tok] = bf16_hi(v.w);
+    }
+    {
+      const int ex = tid >> 2, kq = (tid & 3) * 8;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(w + (size_t)ex * H + k0 + kq));
+      ws[(kq + 0) * WS + ex] = bf16_lo(v.x);
+      ws[(kq + 1) * WS + ex] = bf16_hi(v.x);
+      ws[(kq + 2) * WS + ex] = bf16_lo(v.y);
+      ws[(kq + 3) * WS + ex] = bf16_hi(v.y);
+      ws[(kq + 4) * WS + ex] = bf16_lo(v.z);
+      ws[(kq + 5) * WS + ex] = bf16_hi(v.z);
+      ws[(kq + 6) * WS + ex] = bf16_lo(v.w);
+      ws[(kq + 7) * WS + ex] = bf16_hi(v.w);
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < BK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(xs + kk * XS + ty * 8);
+      const float4 a1 = *reinterpret_cast<const float4*>(xs + kk * XS + ty * 8 + 4);
+      const float4 b = *reinterpret_cast<const float4*>(ws + kk * WS + tx * 4);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* logits = buf;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = tx * 4 + j;
+    const float b = bias != nullptr ? bias[e] : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float v = acc[i][j];
+      if (bias != nullptr) v = __fadd_rn(v, b);
+      logits[(ty * 8 + i) * LS + e] = v;
+    }
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < BT; r += 8) {
+    const int t = t0 + r;
+    if (t < T) topk_softmax_warp<K>(logits + r * LS, lane, idx_out + (size_t)t * K, w_out + (size_t)t * K);
+  }
+}
+
+}  // namespace vg

@@ -1,0 +1,487 @@
+// C ABI of the verifier hot path (declared in include/vgv.h): argument
+// validation, workspace layout, TMA descriptors and kernel launches. One
+// translation unit so the device status word is a single symbol.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "vgv.h"
+#include "common.cuh"
+#include "gemm_moe.cuh"
+#include "lmhead.cuh"
+#include "router.cuh"
+#include "sort.cuh"
+
+namespace {
+
+constexpr int kH = 1280, kI = 896, kE = 64, kS = 2, kTopK = 6;
+constexpr int kMaxDevices = 64;
+constexpr int kSmallRouterMaxT = 512;
+
+struct DevState {
+  bool init = false;
+  int sms = 0;
+};
+DevState g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// ------------------------------------------------------------- timing hook
+struct ProfHook {
+  std::vector<cudaEvent_t> starts, stops;
+  int64_t count = 0;
+};
+ProfHook g_prof[VG_KERNEL_KINDS];
+std::mutex g_prof_mu;
+bool g_prof_any = false;
+
+// Brackets one launch of `kind` with the hook's events, if any are set.
+struct ProfScope {
+  int kind;
+  cudaStream_t s;
+  int64_t slot = -1;
+  ProfScope(int k, cudaStream_t st) : kind(k), s(st) {
+    if (!g_prof_any) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    ProfHook& h = g_prof[kind];
+    if (h.starts.empty()) return;
+    slot = h.count++ % (int64_t)h.starts.size();
+    cudaEventRecord(h.starts[slot], s);
+  }
+  ~ProfScope() {
+    if (slot < 0) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    ProfHook& h = g_prof[kind];
+    if ((int64_t)h.stops.size() > slot) cudaEventRecord(h.stops[slot], s);
+  }
+};
+
+vg_status cuda_fail() {
+  (void)cudaGetLastError();
+  return VG_ERR_CUDA;
+}
+
+// Per-device one-time set-up: SM count, shared-memory opt-in for the big kernels.
+vg_status device_state(DevState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail();
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState& d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cuda_fail();
+    if (cudaFuncSetAttribute(vg::moe_grouped_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::GemmCfg<true>::kSmemBytes) != cudaSuccess)
+      return cuda_fail();
+    if (cudaFuncSetAttribute(vg::moe_grouped_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::GemmCfg<false>::kSmemBytes) != cudaSuccess)
+      return cuda_fail();
+    if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
+        cudaSuccess)
+      return cuda_fail();
+    if (cudaFuncSetAttribute(vg::expert_sort_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::kSortSmallMax * 4) != cudaSuccess)
+      return cuda_fail();
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return cuda_fail();
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.init = true;
+  }
+  *out = &d;
+  return VG_OK;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes.
+vg_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                   const uint32_t* box) {
+  uint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VG_OK : VG_ERR_CUDA;
+}
+
+// Rows of a TMA box: `full`, or the tensor's row count rounded up to 8 when the
+// tensor is shorter than one full box.
+int box_rows(int64_t rows, int full) { return rows >= full ? full : (int)((rows + 7) / 8 * 8); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool dims_supported(const vg_moe_dims* d) {
+  return d->hidden == kH && d->intermediate == kI && d->n_routed == kE && d->n_shared == kS && d->top_k == kTopK;
+}
+
+struct MoeWs {
+  size_t idx, w, offsets, perm, inv, xperm, act, o, ccnt, cbase, total;
+};
+
+MoeWs moe_layout(int T) {
+  const size_t N = (size_t)T * kTopK;
+  const size_t nch = (N + vg::kSortChunk - 1) / vg::kSortChunk;
+  MoeWs L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.idx = take(N * 4);
+  L.w = take(N * 4);
+  L.offsets = take((kE + 1) * 4);
+  L.perm = take(N * 4);
+  L.inv = take(N * 4);
+  L.xperm = take(N * kH * 2);
+  L.act = take((size_t)(kTopK + kS) * T * kI * 2);
+  L.o = take((size_t)(kTopK + kS) * T * kH * 2);
+  L.ccnt = take(nch * kE * 4);
+  L.cbase = take(nch * kE * 4);
+  L.total = off;
+  return L;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Launches one MoE layer; arguments already validated.
+vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, const float* router_bias,
+                     const void* expert_w, const void* shared_w, int add_residual, void* out,
+                     const vg_moe_taps* taps, void* workspace, cudaStream_t s) {
+  using namespace vg;
+  const MoeWs L = moe_layout(T);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = (taps && taps->topk_idx) ? taps->topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* gw = (taps && taps->topk_weight) ? taps->topk_weight : reinterpret_cast<float*>(ws + L.w);
+  int32_t* offsets = (taps && taps->expert_offsets) ? taps->expert_offsets : reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm = (taps && taps->perm) ? taps->perm : reinterpret_cast<int32_t*>(ws + L.perm);
+  int32_t* inv = (taps && taps->inv_perm) ? taps->inv_perm : reinterpret_cast<int32_t*>(ws + L.inv);
+  __nv_bfloat16* xperm = reinterpret_cast<__nv_bfloat16*>(ws + L.xperm);
+  __nv_bfloat16* act = (taps && taps->act) ? static_cast<__nv_bfloat16*>(taps->act) : reinterpret_cast<__nv_bfloat16*>(ws + L.act);
+  __nv_bfloat16* o = (taps && taps->expert_out) ? static_cast<__nv_bfloat16*>(taps->expert_out) : reinterpret_cast<__nv_bfloat16*>(ws + L.o);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  const int N = T * kTopK;
+
+  // 1. router
+  {
+  ProfScope ps(VG_KERNEL_ROUTER, s);
+  if (T <= kSmallRouterMaxT)
+    router_topk_small<kTopK><<<cdiv(T, 4), 256, 0, s>>>(xb, static_cast<const __nv_bfloat16*>(router_w),
+                                                       router_bias, T, kH, idx, gw);
+  else
+    router_topk_tiled<kTopK><<<cdiv(T, 128), 256, 0, s>>>(xb, static_cast<const __nv_bfloat16*>(router_w),
+                                                         router_bias, T, kH, idx, gw);
+  }
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+
+  // 2. grouping by expert + row gather
+  {
+  ProfScope ps(VG_KERNEL_GROUPING, s);
+  if (N <= kSortSmallMax) {
+    const int grid = min(dev->sms, N);
+    expert_sort_small<<<grid, 1024, N * 4, s>>>(idx, N, kTopK, offsets, perm, inv, xb, kH, xperm);
+  } else {
+    const int nch = cdiv(N, kSortChunk);
+    int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
+    int32_t* cbase = reinterpret_cast<int32_t*>(ws + L.cbase);
+    expert_hist_chunks<<<nch, 1024, 0, s>>>(idx, N, ccnt);
+    expert_scan_chunks<<<1, 64, 0, s>>>(ccnt, nch, N, offsets, cbase);
+    expert_scatter_chunks<<<nch, 1024, 0, s>>>(idx, N, kTopK, cbase, perm, inv, xb, kH, xperm);
+  }
+  }
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+
+  // 3. gate/up + SwiGLU (routed experts and the shared ones in one launch)
+  const uint64_t estride = (uint64_t)3 * kI * kH * 2;
+  CUtensorMap mAr, mAs, mBr, mBs;
+  {
+    const uint64_t dA[3] = {kH, 2 * kI, kE}, sA[2] = {kH * 2, estride};
+    const uint64_t dAs[3] = {kH, 2 * kI, kS};
+    const uint32_t bA[3] = {kBK, kBM, 1};
+    const uint64_t dBr[2] = {kH, (uint64_t)N}, sB[1] = {kH * 2};
+    const uint64_t dBs[2] = {kH, (uint64_t)T};
+    const uint32_t bBr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
+    const uint32_t bBs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
+    if (make_map(&mAr, expert_w, 3, dA, sA, bA) || make_map(&mAs, shared_w, 3, dAs, sA, bA) ||
+        make_map(&mBr, xperm, 2, dBr, sB, bBr) || make_map(&mBs, x, 2, dBs, sB, bBs))
+      return VG_ERR_CUDA;
+    GemmArgs a{};
+    a.offsets = offsets;
+    a.T = T;
+    a.E = kE;
+    a.S = kS;
+    a.n_mblk = kI / kBM;
+    a.k_chunks = kH / kBK;
+    a.a_up_row = kI;
+    a.b_shared_base = 0;
+    a.b_shared_stride = 0;
+    a.out_shared_base = N;
+    a.out_ld = kI;
+    a.b_box_r = (int)bBr[1];
+    a.b_box_s = (int)bBs[1];
+    a.out = act;
+    const int units_bound = a.n_mblk * (cdiv(N, kNMax) + kE + kS * cdiv(T, kNMax));
+    const int grid = min(dev->sms, units_bound);
+    ProfScope ps(VG_KERNEL_GATE_UP, s);
+    moe_grouped_gemm<true><<<grid, 192, GemmCfg<true>::kSmemBytes, s>>>(mAr, mAs, mBr, mBs, a);
+    if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  }
+  // 4. down
+  {
+    const __nv_bfloat16* dr = static_cast<const __nv_bfloat16*>(expert_w) + (size_t)2 * kI * kH;
+    const __nv_bfloat16* ds = static_cast<const __nv_bfloat16*>(shared_w) + (size_t)2 * kI * kH;
+    const uint64_t dA[3] = {kI, kH, kE}, sA[2] = {kI * 2, estride};
+    const uint64_t dAs[3] = {kI, kH, kS};
+    const uint32_t bA[3] = {kBK, kBM, 1};
+    const uint64_t dB[2] = {kI, (uint64_t)(kTopK + kS) * T}, sB[1] = {kI * 2};
+    const uint32_t bB[2] = {kBK, (uint32_t)box_rows((kTopK + kS) * T, kBoxRows)};
+    if (make_map(&mAr, dr, 3, dA, sA, bA) || make_map(&mAs, ds, 3, dAs, sA, bA) ||
+        make_map(&mBr, act, 2, dB, sB, bB))
+      return VG_ERR_CUDA;
+    GemmArgs a{};
+    a.offsets = offsets;
+    a.T = T;
+    a.E = kE;
+    a.S = kS;
+    a.n_mblk = kH / kBM;
+    a.k_chunks = kI / kBK;
+    a.a_up_row = 0;
+    a.b_shared_base = N;
+    a.b_shared_stride = T;
+    a.out_shared_base = N;
+    a.out_ld = kH;
+    a.b_box_r = (int)bB[1];
+    a.b_box_s = (int)bB[1];
+    a.out = o;
+    const int units_bound = a.n_mblk * (cdiv(N, kNMax) + kE + kS * cdiv(T, kNMax));
+    const int grid = min(dev->sms, units_bound);
+    ProfScope ps(VG_KERNEL_DOWN, s);
+    moe_grouped_gemm<false><<<grid, 192, GemmCfg<false>::kSmemBytes, s>>>(mAr, mAs, mBr, mBr, a);
+    if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  }
+  // 5. weighted combine + residual
+  {
+    ProfScope ps(VG_KERNEL_COMBINE, s);
+    moe_combine<<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(xb, o, inv, gw, T, kH, kTopK, kS, add_residual,
+                                                       static_cast<__nv_bfloat16*>(out));
+  }
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  return VG_OK;
+}
+
+size_t verify_ws_bytes(int B, int K, int V) {
+  const size_t R = (size_t)B * (K + 1);
+  const size_t nvb = (size_t)vg::cdiv(V, vg::kLmN);
+  return align256(nvb * R * 8);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vg_status_string(vg_status s) {
+  switch (s) {
+    case VG_OK: return "VG_OK";
+    case VG_ERR_INVALID_ARG: return "VG_ERR_INVALID_ARG";
+    case VG_ERR_UNSUPPORTED: return "VG_ERR_UNSUPPORTED";
+    case VG_ERR_WORKSPACE: return "VG_ERR_WORKSPACE";
+    case VG_ERR_CUDA: return "VG_ERR_CUDA";
+    case VG_ERR_TIMEOUT: return "VG_ERR_TIMEOUT";
+    case VG_ERR_DEVICE_BOUNDS: return "VG_ERR_DEVICE_BOUNDS";
+  }
+  return "VG_UNKNOWN";
+}
+
+int32_t vg_abi_version(void) { return 1; }
+
+size_t vg_moe_workspace_bytes(const vg_moe_dims* dims, int32_t T_max) {
+  if (dims == nullptr || !dims_supported(dims) || T_max < 0) return 0;
+  return moe_layout(T_max > 0 ? T_max : 1).total;
+}
+
+static vg_status validate_moe(const vg_moe_dims* dims, int32_t T, const void* x, const void* router_w,
+                              const void* expert_w, const void* shared_w, void* out, void* workspace,
+                              size_t workspace_bytes) {
+  if (dims == nullptr || T < 0) return VG_ERR_INVALID_ARG;
+  if (!dims_supported(dims)) return VG_ERR_UNSUPPORTED;
+  if (T > (1 << 22)) return VG_ERR_UNSUPPORTED;
+  if (T == 0) return VG_OK;
+  if (!x || !router_w || !expert_w || !shared_w || !out) return VG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(router_w) || !aligned16(expert_w) || !aligned16(shared_w) || !aligned16(out))
+    return VG_ERR_INVALID_ARG;
+  const size_t need = moe_layout(T).total;
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return VG_ERR_WORKSPACE;
+  const size_t row_bytes = (size_t)T * kH * 2;
+  if (overlaps(out, row_bytes, x, row_bytes) || overlaps(out, row_bytes, workspace, workspace_bytes))
+    return VG_ERR_INVALID_ARG;
+  return VG_OK;
+}
+
+vg_status vg_moe_ffn(const vg_moe_dims* dims, int32_t T, const void* x, const void* router_w,
+                     const float* router_bias, const void* expert_w, const void* shared_w, int32_t add_residual,
+                     void* out, const vg_moe_taps* taps, void* workspace, size_t workspace_bytes,
+                     vg_stream_t stream) {
+  vg_status st = validate_moe(dims, T, x, router_w, expert_w, shared_w, out, workspace, workspace_bytes);
+  if (st != VG_OK || T == 0) return st;
+  DevState* dev = nullptr;
+  if ((st = device_state(&dev)) != VG_OK) return st;
+  return launch_moe(dev, T, x, router_w, router_bias, expert_w, shared_w, add_residual ? 1 : 0, out, taps,
+                    workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t vg_moe_stack_workspace_bytes(const vg_moe_dims* dims, int32_t T_max) {
+  const size_t m = vg_moe_workspace_bytes(dims, T_max);
+  if (m == 0) return 0;
+  return m + 2 * align256((size_t)(T_max > 0 ? T_max : 1) * kH * 2);
+}
+
+vg_status vg_moe_ffn_stack(const vg_moe_dims* dims, int32_t n_layers, int32_t T, const void* x,
+                           const void* const* router_w, const float* const* router_bias,
+                           const void* const* expert_w, const void* const* shared_w, void* out, void* workspace,
+                           size_t workspace_bytes, vg_stream_t stream) {
+  if (dims == nullptr || n_layers < 1 || T < 0 || !router_w || !expert_w || !shared_w) return VG_ERR_INVALID_ARG;
+  if (!dims_supported(dims)) return VG_ERR_UNSUPPORTED;
+  if (T == 0) return VG_OK;
+  const size_t mw = moe_layout(T).total;
+  const size_t hb = align256((size_t)T * kH * 2);
+  if (workspace == nullptr || workspace_bytes < mw + 2 * hb) return VG_ERR_WORKSPACE;
+  for (int l = 0; l < n_layers; ++l)
+    if (!router_w[l] || !expert_w[l] || !shared_w[l] || !aligned16(router_w[l]) || !aligned16(expert_w[l]) ||
+        !aligned16(shared_w[l]))
+      return VG_ERR_INVALID_ARG;
+  vg_status st = validate_moe(dims, T, x, router_w[0], expert_w[0], shared_w[0], out, workspace, workspace_bytes);
+  if (st != VG_OK) return st;
+  DevState* dev = nullptr;
+  if ((st = device_state(&dev)) != VG_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* buf[2] = {ws + mw, ws + mw + hb};
+  const void* cur = x;
+  for (int l = 0; l < n_layers; ++l) {
+    void* dst = (l == n_layers - 1) ? out : buf[l & 1];
+    st = launch_moe(dev, T, cur, router_w[l], router_bias ? router_bias[l] : nullptr, expert_w[l], shared_w[l], 1,
+                    dst, nullptr, workspace, reinterpret_cast<cudaStream_t>(stream));
+    if (st != VG_OK) return st;
+    cur = dst;
+  }
+  return VG_OK;
+}
+
+size_t vg_verify_workspace_bytes(int32_t B, int32_t K, int32_t H, int32_t V) {
+  if (B < 0 || K < 0 || K > 255 || H != kH || V < 1) return 0;
+  if ((int64_t)B * (K + 1) >= (1 << 24)) return 0;
+  return verify_ws_bytes(B > 0 ? B : 1, K, V);
+}
+
+vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V, const void* h, const void* lm_head,
+                           const int32_t* drafts, int32_t* argmax, int32_t* accepted, int32_t* out_tokens,
+                           void* workspace, size_t workspace_bytes, vg_stream_t stream) {
+  using namespace vg;
+  if (B < 0 || K < 0 || V < 1) return VG_ERR_INVALID_ARG;
+  if (H != kH || K > 255 || (int64_t)B * (K + 1) >= (1 << 24)) return VG_ERR_UNSUPPORTED;
+  if (B == 0) return VG_OK;
+  if (!h || !lm_head || !argmax || !accepted || !out_tokens || (K > 0 && !drafts)) return VG_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(lm_head)) return VG_ERR_INVALID_ARG;
+  const int R = B * (K + 1);
+  if (workspace == nullptr || workspace_bytes < verify_ws_bytes(B, K, V) || !aligned16(workspace))
+    return VG_ERR_WORKSPACE;
+  DevState* dev = nullptr;
+  vg_status st = device_state(&dev);
+  if (st != VG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int n_mblk = cdiv(R, kLmM), n_vblk = cdiv(V, kLmN);
+  const int a_box_rows = box_rows(R, kLmM);
+  CUtensorMap mH, mLM;
+  {
+    const uint64_t dH[2] = {(uint64_t)H, (uint64_t)R}, sH[1] = {(uint64_t)H * 2};
+    const uint32_t bH[2] = {kBK, (uint32_t)a_box_rows};
+    const uint64_t dL[2] = {(uint64_t)H, (uint64_t)V};
+    const uint32_t bL[2] = {kBK, (uint32_t)box_rows(V, kLmN)};
+    if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
+  }
+  uint64_t* part = static_cast<uint64_t*>(workspace);
+  const int grid = min(dev->sms, n_mblk * n_vblk);
+  {
+  ProfScope ps(VG_KERNEL_LM_HEAD, s);
+  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, a_box_rows,
+                                                box_rows(V, kLmN), part);
+  }
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  const int spb = max(1, 32 / (K + 1));
+  {
+    ProfScope ps(VG_KERNEL_ACCEPT, s);
+    argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_vblk, R, B, K, drafts, argmax, accepted, out_tokens);
+  }
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  return VG_OK;
+}
+
+vg_status vg_get_device_status(vg_stream_t stream, int32_t* info) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_fail();
+  int32_t st = 0, inf = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&st, vg::g_status, sizeof(st)) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&inf, vg::g_status_info, sizeof(inf)) != cudaSuccess ||
+      cudaMemcpyToSymbol(vg::g_status, &zero, sizeof(zero)) != cudaSuccess ||
+      cudaMemcpyToSymbol(vg::g_status_info, &zero, sizeof(zero)) != cudaSuccess)
+    return cuda_fail();
+  if (info) *info = inf;
+  return static_cast<vg_status>(st);
+}
+
+vg_status vg_profile_set_events(int32_t kind, const vg_event_t* starts, const vg_event_t* stops, int32_t n) {
+  if (kind < 0 || kind >= VG_KERNEL_KINDS || n < 0 || (n > 0 && (!starts || !stops))) return VG_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (!starts[i] || !stops[i]) return VG_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ProfHook& h = g_prof[kind];
+  h.starts.assign(reinterpret_cast<const cudaEvent_t*>(starts), reinterpret_cast<const cudaEvent_t*>(starts) + n);
+  h.stops.assign(reinterpret_cast<const cudaEvent_t*>(stops), reinterpret_cast<const cudaEvent_t*>(stops) + n);
+  h.count = 0;
+  bool any = false;
+  for (auto& k : g_prof) any = any || !k.starts.empty();
+  g_prof_any = any;
+  return VG_OK;
+}
+
+int64_t vg_profile_count(int32_t kind) {
+  if (kind < 0 || kind >= VG_KERNEL_KINDS) return -1;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_prof[kind].count;
+}
+
+vg_status vg_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) return VG_ERR_INVALID_ARG;
+  if (cudaMemcpyToSymbol(vg::g_wait_timeout_ns, &ns, sizeof(ns)) != cudaSuccess) return cuda_fail();
+  return VG_OK;
+}
+
+}  // extern "C"
+
+namespace vg {
+__global__ void debug_wait_flag_kernel(const int32_t* flag, int32_t expect, uint64_t max_ns) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == expect) return;
+    if (globaltimer() - t0 > max_ns) {
+      record_error(kErrTimeout, 901);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+}  // namespace vg
+
+extern "C" vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uint64_t max_ns, vg_stream_t stream) {
+  if (flag == nullptr || max_ns == 0 || max_ns > 60000000000ull) return VG_ERR_INVALID_ARG;
+  vg::debug_wait_flag_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flag, expect, max_ns);
+  return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}

@@ -1,0 +1,215 @@
+/*
+ * vgv.h — C ABI of the B200 (sm_100a) verifier hot path of jina-ocr-v1's decoder:
+ * the MoE feed-forward layer and the greedy-verify epilogue.
+ *
+ * Sources for what is computed:
+ *  - decoder shape: 12 layers, hidden 1280, 64 routed + 2 shared experts with
+ *    top-6 routing, 129,280-token vocabulary — jina-ocr-v1 model card
+ *    (jina.ai/ko), architecture paragraph; "Jina OCR v1: Быстрый парсинг
+ *    документов на GPU с 24 ГБ VRAM" (aikraft.ru), "01 Архитектура и
+ *    эффективность";
+ *  - six routed experts per token plus two shared ones — "Jina AI's 3.4B OCR
+ *    model targets faster page parsing" (alphasignal.ai), "A compressed visual
+ *    front end";
+ *  - greedy verification, longest agreeing prefix, lossless — "jina-ocr-v1:
+ *    Schnellere Dokumentenanalyse auf kostengünstigen GPUs" (jina.ai/de),
+ *    "Modell und Training"; bonus token counted in tau — same page,
+ *    "Spekulatives Decoding auf einer L4".
+ *
+ * Conventions shared by every call
+ *  - All tensors are caller-owned device memory, row-major, dense. bf16 tensors
+ *    are passed as void*. Pointers must be 16-byte aligned (256-byte aligned
+ *    recommended); the library never allocates, frees or synchronises in the
+ *    compute calls. Calls are asynchronous on the given stream and can be
+ *    captured in a CUDA graph.
+ *  - Every argument is validated before any launch. On a validation error
+ *    nothing is launched and no output is touched.
+ *  - Launch failures return VG_ERR_CUDA. Faults detected on the device (a wait
+ *    that timed out, an index out of range) are recorded in a per-device status
+ *    word read by vg_get_device_status; kernels never trap.
+ *  - The only supported MoE shape is hidden 1280, expert width 896, 64 routed
+ *    experts, 2 shared experts, top-6 (VG_ERR_UNSUPPORTED otherwise). The LM
+ *    head requires hidden 1280 and any vocabulary size 1..2^31-1.
+ *  - T = 0 (or B = 0) is a valid no-op returning VG_OK.
+ */
+#ifndef VGV_H
+#define VGV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* vg_stream_t;
+
+typedef enum vg_status {
+  VG_OK = 0,
+  VG_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, aliasing, misalignment */
+  VG_ERR_UNSUPPORTED = 2,   /* dimensions other than the supported shape */
+  VG_ERR_WORKSPACE = 3,     /* workspace null or smaller than the *_workspace_bytes query */
+  VG_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
+  VG_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (recorded in the status word) */
+  VG_ERR_DEVICE_BOUNDS = 6  /* device: an index check failed (recorded in the status word) */
+} vg_status;
+
+/* MoE layer dimensions: hidden H, expert width I, routed experts E, shared
+ * experts S, experts per token k. Supported: {1280, 896, 64, 2, 6}. */
+typedef struct vg_moe_dims {
+  int32_t hidden;
+  int32_t intermediate;
+  int32_t n_routed;
+  int32_t n_shared;
+  int32_t top_k;
+} vg_moe_dims;
+
+/* Optional views into the layer's intermediates. Each non-NULL pointer is used
+ * by the layer as the storage of that intermediate (so it costs nothing extra);
+ * after the call it holds the value. All are device pointers.
+ *  topk_idx       int32 [T, k]   selected experts, descending router logit,
+ *                                equal logits ordered by lower expert index
+ *  topk_weight    fp32  [T, k]   softmax over all E logits at those experts
+ *  expert_offsets int32 [E + 1]  segment start of each routed expert in the
+ *                                permutation; [E] = T*k
+ *  perm           int32 [T*k]    perm[p] = assignment id t*k + j at position p
+ *                                (stable by assignment id within an expert)
+ *  inv_perm       int32 [T*k]    inv_perm[t*k + j] = its position p
+ *  act            bf16  [(k+S)*T, I]  SwiGLU activations: rows 0..T*k-1 routed
+ *                                in permutation order, row k*T + s*T + t is
+ *                                shared expert s on token t
+ *  expert_out     bf16  [(k+S)*T, H]  unweighted expert outputs, same rows */
+typedef struct vg_moe_taps {
+  int32_t* topk_idx;
+  float* topk_weight;
+  int32_t* expert_offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+  void* act;
+  void* expert_out;
+} vg_moe_taps;
+
+/* Human-readable name of a status code (static storage). */
+const char* vg_status_string(vg_status s);
+
+/* Version of this ABI (incremented on any incompatible change). */
+int32_t vg_abi_version(void);
+
+/* Bytes of workspace vg_moe_ffn needs for up to T_max tokens; 0 if the dims
+ * are unsupported or T_max < 0. */
+size_t vg_moe_workspace_bytes(const vg_moe_dims* dims, int32_t T_max);
+
+/* One MoE feed-forward layer over T tokens.
+ *   logits l[t,e] = fp32 fma chain over h = 0..H-1 of x[t,h]*router_w[e,h]
+ *                   starting at +0, then + router_bias[e] (fp32) if given;
+ *   idx   = the top_k experts by (l descending, e ascending);
+ *   g     = softmax over all E logits at idx (no renormalisation);
+ *   y[t]  = sum_j g[t,j] * SwiGLU_{idx[t,j]}(x[t]) + sum_s SwiGLU^shared_s(x[t]),
+ *           SwiGLU_W(x) = W_down (silu(W_gate x) * (W_up x)), silu(z) = z/(1+e^-z);
+ *   out   = bf16(x + y) if add_residual else bf16(y).
+ * Arguments:
+ *   x            bf16 [T, H]
+ *   router_w     bf16 [E, H]
+ *   router_bias  fp32 [E] or NULL
+ *   expert_w     bf16 [E][gate [I,H] | up [I,H] | down [H,I]], each expert one
+ *                contiguous block of 3*I*H elements
+ *   shared_w     bf16 [S][same layout]
+ *   out          bf16 [T, H]; must not overlap x or the workspace
+ *   taps         NULL or optional intermediate storage (above)
+ *   workspace    device buffer of at least vg_moe_workspace_bytes(dims, T)
+ * Errors: VG_ERR_INVALID_ARG, VG_ERR_UNSUPPORTED, VG_ERR_WORKSPACE, VG_ERR_CUDA. */
+vg_status vg_moe_ffn(const vg_moe_dims* dims, int32_t T,
+                     const void* x, const void* router_w, const float* router_bias,
+                     const void* expert_w, const void* shared_w,
+                     int32_t add_residual, void* out, const vg_moe_taps* taps,
+                     void* workspace, size_t workspace_bytes, vg_stream_t stream);
+
+/* Bytes of workspace vg_moe_ffn_stack needs for up to T_max tokens. */
+size_t vg_moe_stack_workspace_bytes(const vg_moe_dims* dims, int32_t T_max);
+
+/* The decoder's layer loop over its MoE feed-forward layers:
+ * x_{l+1} = bf16(x_l + MoE_l(x_l)) for l = 0..n_layers-1, out = x_{n_layers}.
+ * router_w, router_bias, expert_w, shared_w are HOST arrays of n_layers device
+ * pointers (router_bias may be NULL, or hold NULL entries). out [T,H] must not
+ * overlap x. n_layers >= 1. */
+vg_status vg_moe_ffn_stack(const vg_moe_dims* dims, int32_t n_layers, int32_t T,
+                           const void* x, const void* const* router_w,
+                           const float* const* router_bias,
+                           const void* const* expert_w, const void* const* shared_w,
+                           void* out, void* workspace, size_t workspace_bytes,
+                           vg_stream_t stream);
+
+/* Bytes of workspace vg_verify_greedy needs; 0 if the arguments are invalid. */
+size_t vg_verify_workspace_bytes(int32_t B, int32_t K, int32_t H, int32_t V);
+
+/* Greedy verification of B sequences with K drafted tokens each.
+ *   z[r,v]   = sum_h h[r,h] * lm_head[v,h], accumulated in fp32 on tensor cores
+ *              (never stored);
+ *   argmax[r] = smallest v with z[r,v] = max_v z[r,v];
+ *   accepted[b] = the largest a <= K with drafts[b,i] == argmax[b*(K+1)+i] for
+ *              all i < a;
+ *   out_tokens[b] = drafts[b, 0..a-1], then argmax[b*(K+1)+a] (the bonus
+ *              token), then -1 up to K+1 entries.
+ * Arguments:
+ *   h          bf16 [B*(K+1), H]; row b*(K+1)+i is position i of sequence b
+ *   lm_head    bf16 [V, H]
+ *   drafts     int32 [B, K] (may be NULL when K == 0); drafts[b,i] proposes
+ *              position i+1; values outside [0,V) are valid and never accepted
+ *   argmax     int32 [B*(K+1)]   (out)
+ *   accepted   int32 [B]         (out)
+ *   out_tokens int32 [B, K+1]    (out)
+ *   workspace  device buffer of at least vg_verify_workspace_bytes(B,K,H,V)
+ * H must be 1280; K >= 0; B*(K+1) < 2^24.
+ * Errors: VG_ERR_INVALID_ARG, VG_ERR_UNSUPPORTED, VG_ERR_WORKSPACE, VG_ERR_CUDA. */
+vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V,
+                           const void* h, const void* lm_head, const int32_t* drafts,
+                           int32_t* argmax, int32_t* accepted, int32_t* out_tokens,
+                           void* workspace, size_t workspace_bytes, vg_stream_t stream);
+
+/* Kernel kinds for the timing hook. */
+typedef enum vg_kernel {
+  VG_KERNEL_ROUTER = 0,    /* router logits + top-k + softmax */
+  VG_KERNEL_GROUPING = 1,  /* histogram, stable permutation, row gather */
+  VG_KERNEL_GATE_UP = 2,   /* grouped gate/up GEMM + SwiGLU */
+  VG_KERNEL_DOWN = 3,      /* grouped down GEMM */
+  VG_KERNEL_COMBINE = 4,   /* weighted combine + shared experts + residual */
+  VG_KERNEL_LM_HEAD = 5,   /* LM-head GEMM + per-tile argmax */
+  VG_KERNEL_ACCEPT = 6,    /* argmax reduction + prefix accept */
+  VG_KERNEL_KINDS = 7
+} vg_kernel;
+
+/* Same object as cudaEvent_t. */
+typedef struct CUevent_st* vg_event_t;
+
+/* Timing hook (process-wide, for profiling; no pages' counterpart): while set,
+ * the i-th launch of kernel `kind` counted from this call is bracketed by
+ * cudaEventRecord(starts[i % n]) before it and cudaEventRecord(stops[i % n])
+ * after it, on the stream it is launched on. The events are the caller's
+ * (created with timing enabled) and must outlive the hook. n == 0 clears it.
+ * The arrays are copied; the pointers need not stay valid. */
+vg_status vg_profile_set_events(int32_t kind, const vg_event_t* starts, const vg_event_t* stops, int32_t n);
+
+/* Launches of `kind` recorded since its hook was last set (-1 for a bad kind). */
+int64_t vg_profile_count(int32_t kind);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word: VG_OK if no kernel recorded a fault, else the first recorded code;
+ * *info (if non-NULL) receives a site code of where it happened. */
+vg_status vg_get_device_status(vg_stream_t stream, int32_t* info);
+
+/* Limit, in nanoseconds, for every bounded wait inside the library's kernels on
+ * the current device (default 4 s). Takes effect for launches after the call. */
+vg_status vg_set_wait_timeout_ns(uint64_t ns);
+
+/* Diagnostic: one thread waits (bounded by max_ns) until *flag == expect, using
+ * the same bounded-wait code as the kernels' internal waits. A wait that runs
+ * out records VG_ERR_TIMEOUT in the status word and returns; the context stays
+ * usable. flag is an int32 device pointer. */
+vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uint64_t max_ns,
+                             vg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VGV_H */

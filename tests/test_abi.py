@@ -1,0 +1,117 @@
+"""The C-ABI library builds, loads and exports what include/vgv.h declares;
+host-side validation rejects bad arguments before any CUDA call (CPU only)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import greedy_speculative_verify_b200 as vgv
+from greedy_speculative_verify_b200 import build as vbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    vbuild.build()
+    return vgv.load()
+
+
+def _header_functions(root):
+    src = open(os.path.join(root, "include", "vgv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(vg_[a-z_0-9]+)\s*\(", src))
+
+
+def test_exports_match_header(lib, root_dir):
+    declared = _header_functions(root_dir)
+    assert declared == set(vgv.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", vgv.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T vg_" in l}
+    assert declared <= exported
+
+
+def test_status_strings_and_version(lib):
+    assert vgv.vg_abi_version() == 1
+    for code, name in vgv.STATUS_NAMES.items():
+        assert vgv.vg_status_string(code) == name
+
+
+def test_workspace_queries(lib):
+    d = vgv.MOE_DIMS
+    w128 = vgv.vg_moe_workspace_bytes(d, 128)
+    N = 128 * 6
+    # routing tables, permutation, gathered rows, activations, expert outputs
+    floor = 4 * N * 4 + N * 1280 * 2 + 8 * 128 * 896 * 2 + 8 * 128 * 1280 * 2
+    assert floor <= w128 < floor + 64 * 1024
+    assert vgv.vg_moe_workspace_bytes(d, 256) > w128
+    assert vgv.vg_moe_stack_workspace_bytes(d, 128) >= w128 + 2 * 128 * 1280 * 2
+    assert vgv.vg_moe_workspace_bytes(vgv.vg_moe_dims(1280, 896, 64, 2, 8), 128) == 0
+    assert vgv.vg_moe_workspace_bytes(d, -1) == 0
+    nvb = -(-129280 // 176)
+    assert vgv.vg_verify_workspace_bytes(32, 3, 1280, 129280) >= nvb * 128 * 8
+    assert vgv.vg_verify_workspace_bytes(32, 3, 1024, 129280) == 0
+    assert vgv.vg_verify_workspace_bytes(32, -1, 1280, 129280) == 0
+    assert vgv.vg_verify_workspace_bytes(1 << 22, 3, 1280, 129280) == 0
+
+
+def _moe_call(lib, dims, T, ptrs, ws_bytes, taps=None):
+    x, rw, ew, sw, out, ws = ptrs
+    return lib.vg_moe_ffn(ctypes.byref(dims), T, x, rw, None, ew, sw, 1, out, taps, ws, ws_bytes, None)
+
+
+def test_moe_validation_before_launch(lib):
+    d = vgv.MOE_DIMS
+    A = 1 << 40  # fake, aligned, never dereferenced: validation fails first
+    ok = [A, A + (1 << 30), A + (2 << 30), A + (3 << 30), A + (4 << 30), A + (5 << 30)]
+    need = vgv.vg_moe_workspace_bytes(d, 16)
+    assert _moe_call(lib, d, 0, ok, need) == 0                          # T = 0: no-op
+    assert _moe_call(lib, d, -1, ok, need) == 1                         # negative T
+    assert _moe_call(lib, vgv.vg_moe_dims(1024, 896, 64, 2, 6), 16, ok, need) == 2
+    bad = list(ok); bad[0] = None
+    assert _moe_call(lib, d, 16, bad, need) == 1                        # null x
+    bad = list(ok); bad[2] = A + 8
+    assert _moe_call(lib, d, 16, bad, need) == 1                        # misaligned weights
+    assert _moe_call(lib, d, 16, ok, need - 1) == 3                     # short workspace
+    bad = list(ok); bad[5] = None
+    assert _moe_call(lib, d, 16, bad, need) == 3                        # no workspace
+    bad = list(ok); bad[4] = ok[0] + 64
+    assert _moe_call(lib, d, 16, bad, need) == 1                        # out overlaps x
+
+
+def test_verify_validation_before_launch(lib):
+    A = 1 << 40
+    h, lm, dr, am, ac, ot, ws = (A + (i << 30) for i in range(7))
+    need = vgv.vg_verify_workspace_bytes(4, 3, 1280, 129280)
+    f = lib.vg_verify_greedy
+    assert f(0, 3, 1280, 129280, h, lm, dr, am, ac, ot, ws, need, None) == 0      # B = 0
+    assert f(-1, 3, 1280, 129280, h, lm, dr, am, ac, ot, ws, need, None) == 1
+    assert f(4, -1, 1280, 129280, h, lm, dr, am, ac, ot, ws, need, None) == 1
+    assert f(4, 3, 1280, 0, h, lm, dr, am, ac, ot, ws, need, None) == 1
+    assert f(4, 3, 1024, 129280, h, lm, dr, am, ac, ot, ws, need, None) == 2
+    assert f(4, 3, 1280, 129280, h, lm, None, am, ac, ot, ws, need, None) == 1    # drafts needed for K > 0
+    assert f(4, 3, 1280, 129280, h, None, dr, am, ac, ot, ws, need, None) == 1
+    assert f(4, 3, 1280, 129280, h, lm, dr, am, ac, ot, ws, need - 1, None) == 3
+    assert f(4, 3, 1280, 129280, h + 4, lm, dr, am, ac, ot, ws, need, None) == 1  # misaligned h
+
+
+def test_stack_validation_before_launch(lib):
+    d = vgv.MOE_DIMS
+    arr = ctypes.c_void_p * 2
+    A = 1 << 40
+    rw, ew, sw = arr(A, A), arr(A, A), arr(A, None)
+    need = vgv.vg_moe_stack_workspace_bytes(d, 8)
+    f = lib.vg_moe_ffn_stack
+    assert f(ctypes.byref(d), 0, 8, A, rw, None, ew, sw, A + (1 << 30), A + (2 << 30), need, None) == 1
+    assert f(ctypes.byref(d), 2, 8, A, rw, None, ew, sw, A + (1 << 30), A + (2 << 30), need, None) == 1  # null layer ptr
+    sw = arr(A, A)
+    assert f(ctypes.byref(d), 2, 8, A, rw, None, ew, sw, A + (1 << 30), A + (2 << 30), need - 1, None) == 3
+    assert f(ctypes.byref(d), 2, 0, A, rw, None, ew, sw, A + (1 << 30), A + (2 << 30), need, None) == 0
+
+
+def test_binding_has_no_fallback(tmp_path, monkeypatch):
+    """Without the shared library the binding raises instead of computing."""
+    monkeypatch.setattr(vgv, "_lib", None)
+    monkeypatch.setattr(vgv, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        vgv.vg_abi_version()
