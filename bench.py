@@ -320,6 +320,10 @@ def run_gpu(args, rank, world, local):
     per_step = {k: (1 if k in (vgv.VG_KERNEL_LM_HEAD, vgv.VG_KERNEL_ACCEPT) else LAYERS) for k in kinds}
     evs = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)],
                [torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)]) for k in kinds}
+    for a0, a1 in evs.values():
+        for e in a0 + a1:
+            e.record(stream)  # torch creates the CUDA event at its first record
+    torch.cuda.synchronize()
     for k, (a0, a1) in evs.items():
         vgv.vg_profile_set_events(k, a0, a1)
     for _ in range(kr):
