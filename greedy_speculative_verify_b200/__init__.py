@@ -27,7 +27,7 @@ EXPORTS = (
     "vg_status_string", "vg_abi_version", "vg_moe_workspace_bytes", "vg_moe_ffn",
     "vg_moe_stack_workspace_bytes", "vg_moe_ffn_stack", "vg_verify_workspace_bytes",
     "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag",
-    "vg_profile_set_events", "vg_profile_count",
+    "vg_profile_set_events", "vg_profile_count", "vg_verify_greedy_noalloc",
 )
 
 # vg_kernel
@@ -82,6 +82,7 @@ def load():
         "vg_debug_wait_flag": (i32, [vp, i32, u64, vp]),
         "vg_profile_set_events": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
         "vg_profile_count": (ctypes.c_int64, [i32]),
+        "vg_verify_greedy_noalloc": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -193,3 +194,14 @@ def vg_profile_set_events(kind: int, starts, stops):
 
 def vg_profile_count(kind: int) -> int:
     return load().vg_profile_count(kind)
+
+
+NOALLOC_SCRATCH_KEYS = (2 << 20) // 8
+
+
+def vg_verify_greedy_noalloc(B, K, H, V, h, lm_head, drafts, argmax, accepted, out_tokens, stream=None):
+    """vg_verify_greedy without a workspace, for callers that cannot allocate
+    device memory; see include/vgv.h for the scratch limit and its sharing."""
+    st = load().vg_verify_greedy_noalloc(B, K, H, V, _ptr(h), _ptr(lm_head), _ptr(drafts), _ptr(argmax),
+                                         _ptr(accepted), _ptr(out_tokens), _stream(stream))
+    _check(st, "vg_verify_greedy_noalloc")

@@ -485,3 +485,64 @@ extern "C" vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uin
   vg::debug_wait_flag_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flag, expect, max_ns);
   return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
 }
+
+// ------------------------------------------------------------------ no-alloc
+// Scratch of vg_verify_greedy_noalloc: a file-scope device array (its host-side
+// name is only a stand-in; the device address comes from cudaGetSymbolAddress).
+namespace {
+constexpr size_t kNoAllocKeys = VG_NOALLOC_SCRATCH_BYTES / sizeof(uint64_t);
+static __device__ __align__(256) uint64_t g_noalloc_scratch[kNoAllocKeys];
+uint64_t* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Once per device, with that device current: the array's device address.
+vg_status noalloc_scratch(uint64_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail();
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return cuda_fail();
+    g_noalloc_ptr[dev] = static_cast<uint64_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return VG_OK;
+}
+}  // namespace
+
+extern "C" vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, int32_t V, const void* h,
+                                              const void* lm_head, const int32_t* drafts, int32_t* argmax,
+                                              int32_t* accepted, int32_t* out_tokens, vg_stream_t stream) {
+  using namespace vg;
+  if (B < 0 || K < 0 || V < 1) return VG_ERR_INVALID_ARG;
+  if (H != kH || K > 255 || (int64_t)B * (K + 1) >= (1 << 24)) return VG_ERR_UNSUPPORTED;
+  if (B == 0) return VG_OK;
+  if (!h || !lm_head || !argmax || !accepted || !out_tokens || (K > 0 && !drafts)) return VG_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(lm_head)) return VG_ERR_INVALID_ARG;
+  const int R = B * (K + 1);
+  const int n_mblk = cdiv(R, kLmM), n_vblk = cdiv(V, kLmN);
+  if ((uint64_t)n_vblk * (uint64_t)R > kNoAllocKeys) return VG_ERR_WORKSPACE;
+  DevState* dev = nullptr;
+  vg_status st = device_state(&dev);
+  if (st != VG_OK) return st;
+  uint64_t* part = nullptr;
+  if ((st = noalloc_scratch(&part)) != VG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int a_box_rows = box_rows(R, kLmM);
+  CUtensorMap mH, mLM;
+  {
+    const uint64_t dH[2] = {(uint64_t)H, (uint64_t)R}, sH[1] = {(uint64_t)H * 2};
+    const uint32_t bH[2] = {kBK, (uint32_t)a_box_rows};
+    const uint64_t dL[2] = {(uint64_t)H, (uint64_t)V};
+    const uint32_t bL[2] = {kBK, (uint32_t)box_rows(V, kLmN)};
+    if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
+  }
+  const int grid = min(dev->sms, n_mblk * n_vblk);
+  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, a_box_rows,
+                                                box_rows(V, kLmN), part);
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  const int spb = max(1, 32 / (K + 1));
+  argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_vblk, R, B, K, drafts, argmax, accepted, out_tokens);
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  return VG_OK;
+}

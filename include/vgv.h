@@ -209,6 +209,30 @@ vg_status vg_set_wait_timeout_ns(uint64_t ns);
 vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uint64_t max_ns,
                              vg_stream_t stream);
 
+/* Allocation-free variant of vg_verify_greedy. The pages have no counterpart:
+ * it exists for callers that cannot allocate device memory themselves — a
+ * plugin whose device memory belongs to its host application's pool allocator,
+ * or a latency-critical loop that must not call cudaMalloc because it
+ * synchronises the whole device — and so cannot provide a workspace.
+ * Same computation, arguments and results as vg_verify_greedy, without the
+ * workspace: the per-tile argmax keys go to a scratch array compiled into the
+ * library (VG_NOALLOC_SCRATCH_BYTES = 2 MiB of device memory that every GPU
+ * which loads the library holds until the process exits). Limit:
+ * ceil(V / 176) * B * (K+1) <= VG_NOALLOC_SCRATCH_BYTES / 8 = 262,144 keys
+ * (for V = 129,280: at most 356 verify rows); larger calls return
+ * VG_ERR_WORKSPACE and launch nothing. No call allocates or frees memory.
+ * The first call on each device looks up the scratch array's device address
+ * (with that device current) and caches it; make that first call before any
+ * stream capture. Every call uses the same array: each call overwrites every
+ * key it reads, so nothing needs clearing between calls, but calls whose work
+ * overlaps on the GPU (different streams, or several threads) race on the
+ * array and must be serialised by the caller. */
+#define VG_NOALLOC_SCRATCH_BYTES (2u << 20)
+vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, int32_t V,
+                                   const void* h, const void* lm_head, const int32_t* drafts,
+                                   int32_t* argmax, int32_t* accepted, int32_t* out_tokens,
+                                   vg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
