@@ -48,7 +48,7 @@ WORKLOAD = {
     "B": B, "K": K, "tokens": T, "layers": LAYERS, "vocab": V, "draft_p": P_DRAFT,
     "l2": "inputs larger than L2: 5.78 GB of weights per step vs 126 MB L2, no flush",
 }
-GATE_UP_W_BYTES = 2 * I * H * 2  # gate + up rows of one expert, bf16
+EXPERT_W_BYTES = 3 * I * H * 2  # gate + up + down of one expert, bf16 (6,881,280 B)
 
 
 def _env():
@@ -234,7 +234,7 @@ def run_gpu(args, rank, world, local):
     noise = torch.randint(0, V, (B, K), generator=g, device=dev, dtype=torch.int32)
     drafts.copy_(torch.where(u < P_DRAFT, a, noise))
 
-    # ---- gate/up launch bytes per layer, from each layer's routing (untimed)
+    # ---- expert-GEMM launch bytes per layer, from each layer's routing (untimed)
     n_touched = []
     off = torch.empty(E + 1, dtype=torch.int32, device=dev)
     ws_one = torch.empty(vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device=dev)
@@ -245,8 +245,10 @@ def run_gpu(args, rank, world, local):
         cur, nxt = nxt, cur
     del ws_one
     N = T * TOPK
-    act_bytes = N * H * 2 + T * H * 2 + (N + S * T) * I * 2
-    gate_up_bytes = [(n + S) * GATE_UP_W_BYTES + act_bytes for n in n_touched]
+    # weights of every touched expert and the two shared ones; activations: token
+    # rows read, SwiGLU rows written and read back, expert outputs written
+    act_bytes = N * H * 2 + T * H * 2 + 2 * (N + S * T) * I * 2 + (N + S * T) * H * 2
+    expert_bytes = [(n + S) * EXPERT_W_BYTES + act_bytes for n in n_touched]
 
     # ---- device-timed region: the whole step replayed from a CUDA graph
     step(x, drafts)
@@ -314,9 +316,8 @@ def run_gpu(args, rank, world, local):
 
     # ---- kernel timing: CUDA events around every launch, on the launch stream
     kr = max(1, min(args.steps, 10))
-    kinds = {vgv.VG_KERNEL_ROUTER: "router", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_GATE_UP: "gate_up",
-             vgv.VG_KERNEL_DOWN: "down", vgv.VG_KERNEL_COMBINE: "combine", vgv.VG_KERNEL_LM_HEAD: "lm_head",
-             vgv.VG_KERNEL_ACCEPT: "accept"}
+    kinds = {vgv.VG_KERNEL_ROUTER: "router", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_EXPERTS: "experts",
+             vgv.VG_KERNEL_COMBINE: "combine", vgv.VG_KERNEL_LM_HEAD: "lm_head", vgv.VG_KERNEL_ACCEPT: "accept"}
     per_step = {k: (1 if k in (vgv.VG_KERNEL_LM_HEAD, vgv.VG_KERNEL_ACCEPT) else LAYERS) for k in kinds}
     evs = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)],
                [torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)]) for k in kinds}
@@ -334,8 +335,8 @@ def run_gpu(args, rank, world, local):
         vgv.vg_profile_set_events(k, [], [])
     dur = {k: [s.elapsed_time(e) for s, e in zip(*evs[k])] for k in kinds}
     breakdown = {kinds[k]: sum(dur[k]) / kr for k in kinds}
-    gu = dur[vgv.VG_KERNEL_GATE_UP]
-    gu_bytes = sum(gate_up_bytes[i % LAYERS] for i in range(len(gu)))
+    gu = dur[vgv.VG_KERNEL_EXPERTS]
+    gu_bytes = sum(expert_bytes[i % LAYERS] for i in range(len(gu)))
     achieved = gu_bytes / (sum(gu) / 1e3) / 1e9
     launches_per_step = sum(counts.values()) // kr
     grouping_kernels = 1 if T * TOPK <= 8192 else 3
@@ -367,7 +368,7 @@ def run_gpu(args, rank, world, local):
         "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
-        "roofline": {"bound": "hbm", "kernel": "gate_up (grouped gate/up GEMM + SwiGLU)",
+        "roofline": {"bound": "hbm", "kernel": "moe_expert_gemms (gate/up + SwiGLU + down, routed + shared)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
                      "algorithmic_bytes_per_launch": gu_bytes / max(1, len(gu)),

@@ -31,8 +31,8 @@ EXPORTS = (
 )
 
 # vg_kernel
-VG_KERNEL_ROUTER, VG_KERNEL_GROUPING, VG_KERNEL_GATE_UP, VG_KERNEL_DOWN = 0, 1, 2, 3
-VG_KERNEL_COMBINE, VG_KERNEL_LM_HEAD, VG_KERNEL_ACCEPT = 4, 5, 6
+VG_KERNEL_ROUTER, VG_KERNEL_GROUPING, VG_KERNEL_EXPERTS = 0, 1, 2
+VG_KERNEL_COMBINE, VG_KERNEL_LM_HEAD, VG_KERNEL_ACCEPT = 3, 4, 5
 
 
 class VgError(RuntimeError):

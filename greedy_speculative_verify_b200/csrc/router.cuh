@@ -78,30 +78,72 @@ __device__ __forceinline__ void topk_softmax_warp(const float* l, int lane, int3
 }
 
 // Small token counts: one thread per (token, expert) output, 4 tokens x 64
-// experts per block; operands stream from L1/L2 with 16-byte loads.
+// experts per block. The router weights and the 4 token rows stream through
+// shared memory in 128-element chunks with cp.async double buffering, so the
+// only latency left on the critical path is the fma chain itself.
+constexpr int kRtChunk = 128;               // k per chunk
+constexpr int kRtWStride = kRtChunk + 8;    // padded row (272 B): conflict-free 16-byte reads
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int K>
 __global__ void __launch_bounds__(256) router_topk_small(const __nv_bfloat16* __restrict__ x,
                                                          const __nv_bfloat16* __restrict__ w,
                                                          const float* __restrict__ bias, int T, int H,
                                                          int32_t* __restrict__ idx_out,
                                                          float* __restrict__ w_out) {
+  __shared__ __align__(16) __nv_bfloat16 ws[2][kRouterE * kRtWStride];
+  __shared__ __align__(16) __nv_bfloat16 xs[2][4 * kRtChunk];
   __shared__ float logit[4][kRouterE];
-  const int tl = threadIdx.x >> 6, e = threadIdx.x & 63;
-  const int t = blockIdx.x * 4 + tl;
+  const int tid = threadIdx.x;
+  const int tl = tid >> 6, e = tid & 63;
+  const int t0 = blockIdx.x * 4;
+  const int nchunks = H / kRtChunk;
+
+  auto load_chunk = [&](int c, int buf) {
+    const int k0 = c * kRtChunk;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // 64 rows x 16 pieces of 16 B
+      const int q = tid + i * 256;
+      const int row = q >> 4, piece = q & 15;
+      cp_async16(&ws[buf][row * kRtWStride + piece * 8], w + (size_t)row * H + k0 + piece * 8);
+    }
+    if (tid < 64) {  // 4 token rows x 16 pieces
+      const int row = tid >> 4, piece = tid & 15;
+      const int t = min(t0 + row, T - 1);
+      cp_async16(&xs[buf][row * kRtChunk + piece * 8], x + (size_t)t * H + k0 + piece * 8);
+    }
+    cp_async_commit();
+  };
+
   float acc = 0.0f;
-  if (t < T) {
-    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    const uint4* wr = reinterpret_cast<const uint4*>(w + (size_t)e * H);
-    const int nc = H / 8;
-#pragma unroll 4
-    for (int c = 0; c < nc; ++c) fma8(acc, __ldg(xr + c), __ldg(wr + c));
-    if (bias != nullptr) acc = __fadd_rn(acc, bias[e]);
+  load_chunk(0, 0);
+  for (int c = 0; c < nchunks; ++c) {
+    const int buf = c & 1;
+    if (c + 1 < nchunks) {
+      load_chunk(c + 1, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint4* wr = reinterpret_cast<const uint4*>(&ws[buf][e * kRtWStride]);
+    const uint4* xr = reinterpret_cast<const uint4*>(&xs[buf][tl * kRtChunk]);
+#pragma unroll
+    for (int p = 0; p < kRtChunk / 8; ++p) fma8(acc, xr[p], wr[p]);
+    __syncthreads();
   }
+  if (bias != nullptr) acc = __fadd_rn(acc, bias[e]);
   logit[tl][e] = acc;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = tid >> 5, lane = tid & 31;
   if (warp < 4) {
-    const int tt = blockIdx.x * 4 + warp;
+    const int tt = t0 + warp;
     if (tt < T) topk_softmax_warp<K>(logit[warp], lane, idx_out + (size_t)tt * K, w_out + (size_t)tt * K);
   }
 }

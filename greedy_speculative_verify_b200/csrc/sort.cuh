@@ -88,12 +88,15 @@ __global__ void __launch_bounds__(1024) expert_sort_small(const int32_t* __restr
                                                           int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                                                           const __nv_bfloat16* __restrict__ x, int H,
-                                                          __nv_bfloat16* __restrict__ x_perm) {
+                                                          __nv_bfloat16* __restrict__ x_perm,
+                                                          int32_t* __restrict__ sched, int sched_len) {
   extern __shared__ int32_t perm_s[];  // [N]
   __shared__ int cnt[kSortE], run[kSortE];
   __shared__ int wcnt[32][kSortE];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid < kSortE) cnt[tid] = 0;
+  if (blockIdx.x == 0)  // the expert GEMMs' ticket counter and per-tile readiness words
+    for (int i = tid; i < sched_len; i += blockDim.x) sched[i] = 0;
   __syncthreads();
   for (int a = tid; a < N; a += blockDim.x) {
     const int key = keys[a];
@@ -143,9 +146,11 @@ __global__ void __launch_bounds__(1024) expert_hist_chunks(const int32_t* __rest
 // Pass 2 (one block of 64 threads): offsets and each chunk's per-expert base.
 __global__ void __launch_bounds__(64) expert_scan_chunks(const int32_t* __restrict__ chunk_cnt, int nchunks, int N,
                                                          int32_t* __restrict__ offsets,
-                                                         int32_t* __restrict__ chunk_base) {
+                                                         int32_t* __restrict__ chunk_base,
+                                                         int32_t* __restrict__ sched, int sched_len) {
   __shared__ int tot[kSortE], off[kSortE];
   const int e = threadIdx.x;
+  for (int i = e; i < sched_len; i += blockDim.x) sched[i] = 0;  // expert GEMM tickets + readiness
   int s = 0;
   for (int c = 0; c < nchunks; ++c) s += chunk_cnt[c * kSortE + e];
   tot[e] = s;

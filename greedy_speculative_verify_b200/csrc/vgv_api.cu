@@ -71,11 +71,8 @@ vg_status device_state(DevState** out) {
   DevState& d = g_dev[dev];
   if (!d.init) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cuda_fail();
-    if (cudaFuncSetAttribute(vg::moe_grouped_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::GemmCfg<true>::kSmemBytes) != cudaSuccess)
-      return cuda_fail();
-    if (cudaFuncSetAttribute(vg::moe_grouped_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::GemmCfg<false>::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(vg::moe_expert_gemms, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::kFgSmemBytes) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
@@ -120,8 +117,13 @@ bool dims_supported(const vg_moe_dims* d) {
 }
 
 struct MoeWs {
-  size_t idx, w, offsets, perm, inv, xperm, act, o, ccnt, cbase, total;
+  size_t idx, w, offsets, perm, inv, xperm, act, o, ccnt, cbase, sched, total;
+  int sched_len;
 };
+
+// Upper bound of the expert GEMMs' token tiles: routed segments cut at 128 plus
+// one partial tile per routed expert, plus the shared experts' tiles.
+int max_tiles(int T) { return vg::cdiv(T * kTopK, vg::kNMax) + kE + kS * vg::cdiv(T, vg::kNMax); }
 
 MoeWs moe_layout(int T) {
   const size_t N = (size_t)T * kTopK;
@@ -143,6 +145,8 @@ MoeWs moe_layout(int T) {
   L.o = take((size_t)(kTopK + kS) * T * kH * 2);
   L.ccnt = take(nch * kE * 4);
   L.cbase = take(nch * kE * 4);
+  L.sched_len = 1 + max_tiles(T);
+  L.sched = take((size_t)L.sched_len * 4);
   L.total = off;
   return L;
 }
@@ -169,6 +173,7 @@ vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, 
   __nv_bfloat16* o = (taps && taps->expert_out) ? static_cast<__nv_bfloat16*>(taps->expert_out) : reinterpret_cast<__nv_bfloat16*>(ws + L.o);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   const int N = T * kTopK;
+  int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
 
   // 1. router
   {
@@ -187,84 +192,57 @@ vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, 
   ProfScope ps(VG_KERNEL_GROUPING, s);
   if (N <= kSortSmallMax) {
     const int grid = min(dev->sms, N);
-    expert_sort_small<<<grid, 1024, N * 4, s>>>(idx, N, kTopK, offsets, perm, inv, xb, kH, xperm);
+    expert_sort_small<<<grid, 1024, N * 4, s>>>(idx, N, kTopK, offsets, perm, inv, xb, kH, xperm, sched,
+                                                L.sched_len);
   } else {
     const int nch = cdiv(N, kSortChunk);
     int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
     int32_t* cbase = reinterpret_cast<int32_t*>(ws + L.cbase);
     expert_hist_chunks<<<nch, 1024, 0, s>>>(idx, N, ccnt);
-    expert_scan_chunks<<<1, 64, 0, s>>>(ccnt, nch, N, offsets, cbase);
+    expert_scan_chunks<<<1, 64, 0, s>>>(ccnt, nch, N, offsets, cbase, sched, L.sched_len);
     expert_scatter_chunks<<<nch, 1024, 0, s>>>(idx, N, kTopK, cbase, perm, inv, xb, kH, xperm);
   }
   }
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
 
-  // 3. gate/up + SwiGLU (routed experts and the shared ones in one launch)
-  const uint64_t estride = (uint64_t)3 * kI * kH * 2;
-  CUtensorMap mAr, mAs, mBr, mBs;
+  // 3. expert GEMMs: gate/up + SwiGLU then down, routed and shared experts, one launch
   {
-    const uint64_t dA[3] = {kH, 2 * kI, kE}, sA[2] = {kH * 2, estride};
-    const uint64_t dAs[3] = {kH, 2 * kI, kS};
-    const uint32_t bA[3] = {kBK, kBM, 1};
-    const uint64_t dBr[2] = {kH, (uint64_t)N}, sB[1] = {kH * 2};
-    const uint64_t dBs[2] = {kH, (uint64_t)T};
-    const uint32_t bBr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
-    const uint32_t bBs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
-    if (make_map(&mAr, expert_w, 3, dA, sA, bA) || make_map(&mAs, shared_w, 3, dAs, sA, bA) ||
-        make_map(&mBr, xperm, 2, dBr, sB, bBr) || make_map(&mBs, x, 2, dBs, sB, bBs))
-      return VG_ERR_CUDA;
-    GemmArgs a{};
-    a.offsets = offsets;
-    a.T = T;
-    a.E = kE;
-    a.S = kS;
-    a.n_mblk = kI / kBM;
-    a.k_chunks = kH / kBK;
-    a.a_up_row = kI;
-    a.b_shared_base = 0;
-    a.b_shared_stride = 0;
-    a.out_shared_base = N;
-    a.out_ld = kI;
-    a.b_box_r = (int)bBr[1];
-    a.b_box_s = (int)bBs[1];
-    a.out = act;
-    const int units_bound = a.n_mblk * (cdiv(N, kNMax) + kE + kS * cdiv(T, kNMax));
-    const int grid = min(dev->sms, units_bound);
-    ProfScope ps(VG_KERNEL_GATE_UP, s);
-    moe_grouped_gemm<true><<<grid, 192, GemmCfg<true>::kSmemBytes, s>>>(mAr, mAs, mBr, mBs, a);
-    if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
-  }
-  // 4. down
-  {
+    const uint64_t estride = (uint64_t)3 * kI * kH * 2;
     const __nv_bfloat16* dr = static_cast<const __nv_bfloat16*>(expert_w) + (size_t)2 * kI * kH;
-    const __nv_bfloat16* ds = static_cast<const __nv_bfloat16*>(shared_w) + (size_t)2 * kI * kH;
-    const uint64_t dA[3] = {kI, kH, kE}, sA[2] = {kI * 2, estride};
-    const uint64_t dAs[3] = {kI, kH, kS};
+    const __nv_bfloat16* dsh = static_cast<const __nv_bfloat16*>(shared_w) + (size_t)2 * kI * kH;
+    CUtensorMap mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct;
+    const uint64_t dGu[3] = {kH, 2 * kI, kE}, dGuS[3] = {kH, 2 * kI, kS}, sGu[2] = {kH * 2, estride};
+    const uint64_t dDn[3] = {kI, kH, kE}, dDnS[3] = {kI, kH, kS}, sDn[2] = {kI * 2, estride};
     const uint32_t bA[3] = {kBK, kBM, 1};
-    const uint64_t dB[2] = {kI, (uint64_t)(kTopK + kS) * T}, sB[1] = {kI * 2};
-    const uint32_t bB[2] = {kBK, (uint32_t)box_rows((kTopK + kS) * T, kBoxRows)};
-    if (make_map(&mAr, dr, 3, dA, sA, bA) || make_map(&mAs, ds, 3, dAs, sA, bA) ||
-        make_map(&mBr, act, 2, dB, sB, bB))
+    const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
+    const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
+    const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
+    const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
+    const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, kBoxRows)};
+    if (make_map(&mGuR, expert_w, 3, dGu, sGu, bA) || make_map(&mGuS, shared_w, 3, dGuS, sGu, bA) ||
+        make_map(&mDnR, dr, 3, dDn, sDn, bA) || make_map(&mDnS, dsh, 3, dDnS, sDn, bA) ||
+        make_map(&mXr, xperm, 2, dXr, sX, bXr) || make_map(&mXs, x, 2, dXs, sX, bXs) ||
+        make_map(&mAct, act, 2, dAct, sAct, bAct))
       return VG_ERR_CUDA;
-    GemmArgs a{};
+    FusedArgs a{};
     a.offsets = offsets;
     a.T = T;
     a.E = kE;
     a.S = kS;
-    a.n_mblk = kH / kBM;
-    a.k_chunks = kI / kBK;
-    a.a_up_row = 0;
-    a.b_shared_base = N;
-    a.b_shared_stride = T;
-    a.out_shared_base = N;
-    a.out_ld = kH;
-    a.b_box_r = (int)bB[1];
-    a.b_box_s = (int)bB[1];
+    a.mblk_gu = kI / kBM;
+    a.mblk_dn = kH / kBM;
+    a.kc_gu = kH / kBK;
+    a.kc_dn = kI / kBK;
+    a.a_up_row = kI;
+    a.box_xr = (int)bXr[1];
+    a.box_xs = (int)bXs[1];
+    a.box_act = (int)bAct[1];
+    a.sched = sched;
+    a.act = act;
     a.out = o;
-    const int units_bound = a.n_mblk * (cdiv(N, kNMax) + kE + kS * cdiv(T, kNMax));
-    const int grid = min(dev->sms, units_bound);
-    ProfScope ps(VG_KERNEL_DOWN, s);
-    moe_grouped_gemm<false><<<grid, 192, GemmCfg<false>::kSmemBytes, s>>>(mAr, mAs, mBr, mBr, a);
+    const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
+    ProfScope ps(VG_KERNEL_EXPERTS, s);
+    moe_expert_gemms<<<grid, 192, kFgSmemBytes, s>>>(mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct, a);
     if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   }
   // 5. weighted combine + residual
@@ -279,8 +257,8 @@ vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, 
 
 size_t verify_ws_bytes(int B, int K, int V) {
   const size_t R = (size_t)B * (K + 1);
-  const size_t nvb = (size_t)vg::cdiv(V, vg::kLmN);
-  return align256(nvb * R * 8);
+  const size_t ng = (size_t)vg::cdiv(vg::cdiv(V, vg::kLmN), vg::kLmGroupTiles);
+  return align256(ng * R * 8);
 }
 
 }  // namespace
@@ -300,7 +278,7 @@ const char* vg_status_string(vg_status s) {
   return "VG_UNKNOWN";
 }
 
-int32_t vg_abi_version(void) { return 1; }
+int32_t vg_abi_version(void) { return 2; }
 
 size_t vg_moe_workspace_bytes(const vg_moe_dims* dims, int32_t T_max) {
   if (dims == nullptr || !dims_supported(dims) || T_max < 0) return 0;
@@ -407,17 +385,18 @@ vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V, const voi
     if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
   }
   uint64_t* part = static_cast<uint64_t*>(workspace);
-  const int grid = min(dev->sms, n_mblk * n_vblk);
+  const int n_groups = cdiv(n_vblk, kLmGroupTiles);
+  const int grid = min(dev->sms, n_mblk * n_groups);
   {
   ProfScope ps(VG_KERNEL_LM_HEAD, s);
-  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, a_box_rows,
-                                                box_rows(V, kLmN), part);
+  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, kLmGroupTiles, n_groups,
+                                                a_box_rows, box_rows(V, kLmN), part);
   }
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   const int spb = max(1, 32 / (K + 1));
   {
     ProfScope ps(VG_KERNEL_ACCEPT, s);
-    argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_vblk, R, B, K, drafts, argmax, accepted, out_tokens);
+    argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_groups, R, B, K, drafts, argmax, accepted, out_tokens);
   }
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   return VG_OK;
@@ -521,7 +500,8 @@ extern "C" vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, i
   if (!aligned16(h) || !aligned16(lm_head)) return VG_ERR_INVALID_ARG;
   const int R = B * (K + 1);
   const int n_mblk = cdiv(R, kLmM), n_vblk = cdiv(V, kLmN);
-  if ((uint64_t)n_vblk * (uint64_t)R > kNoAllocKeys) return VG_ERR_WORKSPACE;
+  const int n_groups = cdiv(n_vblk, kLmGroupTiles);
+  if ((uint64_t)n_groups * (uint64_t)R > kNoAllocKeys) return VG_ERR_WORKSPACE;
   DevState* dev = nullptr;
   vg_status st = device_state(&dev);
   if (st != VG_OK) return st;
@@ -537,12 +517,12 @@ extern "C" vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, i
     const uint32_t bL[2] = {kBK, (uint32_t)box_rows(V, kLmN)};
     if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
   }
-  const int grid = min(dev->sms, n_mblk * n_vblk);
-  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, a_box_rows,
-                                                box_rows(V, kLmN), part);
+  const int grid = min(dev->sms, n_mblk * n_groups);
+  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, kLmGroupTiles, n_groups,
+                                                a_box_rows, box_rows(V, kLmN), part);
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   const int spb = max(1, 32 / (K + 1));
-  argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_vblk, R, B, K, drafts, argmax, accepted, out_tokens);
+  argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_groups, R, B, K, drafts, argmax, accepted, out_tokens);
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   return VG_OK;
 }

@@ -171,12 +171,11 @@ vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V,
 typedef enum vg_kernel {
   VG_KERNEL_ROUTER = 0,    /* router logits + top-k + softmax */
   VG_KERNEL_GROUPING = 1,  /* histogram, stable permutation, row gather */
-  VG_KERNEL_GATE_UP = 2,   /* grouped gate/up GEMM + SwiGLU */
-  VG_KERNEL_DOWN = 3,      /* grouped down GEMM */
-  VG_KERNEL_COMBINE = 4,   /* weighted combine + shared experts + residual */
-  VG_KERNEL_LM_HEAD = 5,   /* LM-head GEMM + per-tile argmax */
-  VG_KERNEL_ACCEPT = 6,    /* argmax reduction + prefix accept */
-  VG_KERNEL_KINDS = 7
+  VG_KERNEL_EXPERTS = 2,   /* expert GEMMs: gate/up + SwiGLU, then down (one launch) */
+  VG_KERNEL_COMBINE = 3,   /* weighted combine + shared experts + residual */
+  VG_KERNEL_LM_HEAD = 4,   /* LM-head GEMM + per-tile argmax */
+  VG_KERNEL_ACCEPT = 5,    /* argmax reduction + prefix accept */
+  VG_KERNEL_KINDS = 6
 } vg_kernel;
 
 /* Same object as cudaEvent_t. */
@@ -217,9 +216,10 @@ vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uint64_t max_n
  * Same computation, arguments and results as vg_verify_greedy, without the
  * workspace: the per-tile argmax keys go to a scratch array compiled into the
  * library (VG_NOALLOC_SCRATCH_BYTES = 2 MiB of device memory that every GPU
- * which loads the library holds until the process exits). Limit:
- * ceil(V / 176) * B * (K+1) <= VG_NOALLOC_SCRATCH_BYTES / 8 = 262,144 keys
- * (for V = 129,280: at most 356 verify rows); larger calls return
+ * which loads the library holds until the process exits). Limit: one key per
+ * (group of 5 vocabulary tiles of 176 rows, verify row),
+ * ceil(ceil(V / 176) / 5) * B * (K+1) <= VG_NOALLOC_SCRATCH_BYTES / 8 = 262,144
+ * keys (for V = 129,280: at most 1,783 verify rows); larger calls return
  * VG_ERR_WORKSPACE and launch nothing. No call allocates or frees memory.
  * The first call on each device looks up the scratch array's device address
  * (with that device current) and caches it; make that first call before any

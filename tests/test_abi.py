@@ -32,7 +32,7 @@ def test_exports_match_header(lib, root_dir):
 
 
 def test_status_strings_and_version(lib):
-    assert vgv.vg_abi_version() == 1
+    assert vgv.vg_abi_version() == 2
     for code, name in vgv.STATUS_NAMES.items():
         assert vgv.vg_status_string(code) == name
 
@@ -48,8 +48,8 @@ def test_workspace_queries(lib):
     assert vgv.vg_moe_stack_workspace_bytes(d, 128) >= w128 + 2 * 128 * 1280 * 2
     assert vgv.vg_moe_workspace_bytes(vgv.vg_moe_dims(1280, 896, 64, 2, 8), 128) == 0
     assert vgv.vg_moe_workspace_bytes(d, -1) == 0
-    nvb = -(-129280 // 176)
-    assert vgv.vg_verify_workspace_bytes(32, 3, 1280, 129280) >= nvb * 128 * 8
+    groups = -(-(-(-129280 // 176)) // 5)  # 5 vocabulary tiles of 176 rows per key
+    assert vgv.vg_verify_workspace_bytes(32, 3, 1280, 129280) >= groups * 128 * 8
     assert vgv.vg_verify_workspace_bytes(32, 3, 1024, 129280) == 0
     assert vgv.vg_verify_workspace_bytes(32, -1, 1280, 129280) == 0
     assert vgv.vg_verify_workspace_bytes(1 << 22, 3, 1280, 129280) == 0

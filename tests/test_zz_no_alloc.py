@@ -61,13 +61,13 @@ def test_noalloc_matches_workspace_entry_two_calls():
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
-    """ceil(V/176) * B*(K+1) keys must fit the 2 MiB array; a larger call
-    returns VG_ERR_WORKSPACE before any CUDA call (so this runs without a GPU)."""
-    vgv.load()
+    """ceil(ceil(V/176)/5) * B*(K+1) keys must fit the 2 MiB array; a larger
+    call returns VG_ERR_WORKSPACE before any CUDA call (so this runs without a
+    GPU)."""
     lib = vgv.load()
     A = 1 << 40
-    nvb = -(-D.V // 176)
-    R_max = vgv.NOALLOC_SCRATCH_KEYS // nvb
+    groups = -(-(-(-D.V // 176)) // 5)
+    R_max = vgv.NOALLOC_SCRATCH_KEYS // groups
     B_bad = R_max // 4 + 1  # K = 3 -> 4 rows per sequence, just past the limit
     assert lib.vg_verify_greedy_noalloc(B_bad, 3, D.H, D.V, A, A, A, A, A, A, None) == 3
     assert lib.vg_verify_greedy_noalloc(0, 3, D.H, D.V, A, A, A, A, A, A, None) == 0
