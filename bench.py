@@ -314,33 +314,39 @@ def run_gpu(args, rank, world, local):
     h2d = x_host.numel() * x_host.element_size() + d_host.numel() * d_host.element_size()
     d2h = acc_host.numel() * acc_host.element_size() + tok_host.numel() * tok_host.element_size()
 
-    # ---- kernel timing: CUDA events around every launch, on the launch stream
+    # ---- kernel timing: CUDA events around every launch, on the launch stream.
+    # One step is captured with the library's timing hook set, so every launch
+    # is bracketed by event-record nodes; each replay is read before the next.
     kr = max(1, min(args.steps, 10))
-    kinds = {vgv.VG_KERNEL_ROUTER: "router", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_EXPERTS: "experts",
+    kinds = {vgv.VG_KERNEL_ROUTER: "layer_entry", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_EXPERTS: "experts",
              vgv.VG_KERNEL_COMBINE: "combine", vgv.VG_KERNEL_LM_HEAD: "lm_head", vgv.VG_KERNEL_ACCEPT: "accept"}
-    per_step = {k: (1 if k in (vgv.VG_KERNEL_LM_HEAD, vgv.VG_KERNEL_ACCEPT) else LAYERS) for k in kinds}
-    evs = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)],
-               [torch.cuda.Event(enable_timing=True) for _ in range(per_step[k] * kr)]) for k in kinds}
+    cap = LAYERS + 1  # no kind launches more often than this in one step
+    evs = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(cap)],
+               [torch.cuda.Event(enable_timing=True) for _ in range(cap)]) for k in kinds}
     for a0, a1 in evs.values():
         for e in a0 + a1:
             e.record(stream)  # torch creates the CUDA event at its first record
     torch.cuda.synchronize()
     for k, (a0, a1) in evs.items():
         vgv.vg_profile_set_events(k, a0, a1)
-    for _ in range(kr):
+    pgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pgraph):
         step(x, drafts)
-    torch.cuda.synchronize()
-    counts = {k: vgv.vg_profile_count(k) for k in kinds}
+    counts = {k: vgv.vg_profile_count(k) for k in kinds}  # launches of each kind in one step
     for k in kinds:
         vgv.vg_profile_set_events(k, [], [])
-    dur = {k: [s.elapsed_time(e) for s, e in zip(*evs[k])] for k in kinds}
-    breakdown = {kinds[k]: sum(dur[k]) / kr for k in kinds}
+    dur = {k: [] for k in kinds}
+    for _ in range(kr):
+        pgraph.replay()
+        torch.cuda.synchronize()
+        for k, (a0, a1) in evs.items():
+            dur[k].extend(s.elapsed_time(e) for s, e in zip(a0[:counts[k]], a1[:counts[k]]))
+    del pgraph
+    breakdown = {kinds[k]: sum(dur[k]) / kr for k in kinds if dur[k]}
     gu = dur[vgv.VG_KERNEL_EXPERTS]
     gu_bytes = sum(expert_bytes[i % LAYERS] for i in range(len(gu)))
     achieved = gu_bytes / (sum(gu) / 1e3) / 1e9
-    launches_per_step = sum(counts.values()) // kr
-    grouping_kernels = 1 if T * TOPK <= 8192 else 3
-    launches_per_step += (grouping_kernels - 1) * LAYERS
+    launches_per_step = sum(counts.values())
 
     # ---- aggregate over ranks (max time, summed tokens)
     if world > 1:

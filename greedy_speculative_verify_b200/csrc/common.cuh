@@ -108,6 +108,15 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
       : "memory");
 }
+// Plain (untiled) bulk copy global -> shared, completing on an mbarrier. Both
+// addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -192,6 +201,37 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- grid barrier
+// Barrier over all CTAs of a cooperative launch, on one counter that only grows:
+// every CTA adds 1 (a fire-and-forget release reduction, so arrivals do not
+// serialise on a round trip) and waits until the counter reaches `target`
+// = (number of barriers passed on this counter since it was zeroed + 1) * CTAs.
+// Bounded: returns false (and records VG_ERR_TIMEOUT) if the limit runs out.
+__device__ __forceinline__ bool grid_barrier(uint32_t* ctr, uint32_t target, uint64_t limit_ns, int32_t site) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();  // this CTA's writes (ordered before by __syncthreads) precede the arrival
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+    const uint64_t t0 = globaltimer();
+    while (true) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if ((int32_t)(v - target) >= 0) break;
+      if (globaltimer() - t0 > limit_ns) {
+        record_error(kErrTimeout, site);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
 }
 
 // ----------------------------------------------------------------- misc

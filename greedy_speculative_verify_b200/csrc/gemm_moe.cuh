@@ -38,18 +38,28 @@ namespace vg {
 
 constexpr int kBM = 128;       // weight rows per tile
 constexpr int kBK = 64;        // K elements per stage: one 128-byte swizzle row
-constexpr int kNMax = 128;     // tokens per tile
+constexpr int kNMax = 128;     // tokens per tile, widest configuration
 constexpr int kBoxRows = 16;   // token rows per TMA box of the B operand
 constexpr int kMaxExperts = 72;
 
-constexpr int kFgStages = 4;
-constexpr int kFgABytes = kBM * kBK * 2;                  // 16 KB
-constexpr int kFgBBytes = kNMax * kBK * 2;                // 16 KB
-constexpr int kFgStageBytes = 2 * kFgABytes + kFgBBytes;  // A_gate | A_up (or A_down) | B
-constexpr int kFgAccCols = 2 * kNMax;                     // one accumulator buffer (gate | up)
-constexpr int kFgTmemCols = 2 * kFgAccCols;               // double buffered: 512
-constexpr int kFgAuxBytes = 2048;
-constexpr int kFgSmemBytes = kFgStages * kFgStageBytes + kFgAuxBytes + 1024;  // + alignment slack
+// Two configurations of the same kernel, by tile width NMAX:
+//  * NMAX = 128, 4 stages: prefill-sized expert segments, 128 x 128 tiles;
+//  * NMAX = 64, 5 stages: decode sizes, where the token slot of a stage is
+//    small and the freed shared memory buys a fifth stage of weights in flight.
+// A stage holds two 16 KB weight tiles and an NMAX x 64 token slot.
+template <int NMAX>
+struct FgCfg {
+  static constexpr int kStages = NMAX == 128 ? 4 : 5;
+  static constexpr int kABytes = kBM * kBK * 2;          // 16 KB
+  static constexpr int kBBytes = NMAX * kBK * 2;         // token slot
+  static constexpr int kStageBytes = 2 * kABytes + kBBytes;
+  static constexpr int kAccCols = 2 * NMAX;              // one accumulator buffer (gate | up)
+  static constexpr int kTmemCols = 2 * kAccCols;         // double buffered
+  static constexpr int kAuxBytes = 2048;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kAuxBytes + 1024;  // + alignment slack
+  static constexpr int kPairBOff = kBBytes / 2;          // second k-chunk's token rows in a paired stage
+};
+constexpr int kFgABytes = kBM * kBK * 2;
 constexpr int kFgRing = 4;                                // unit-ticket ring between the roles
 constexpr int kFgEpiWarps = 4;
 
@@ -79,7 +89,7 @@ struct FgUnit {
   int tile, e, mb, nrows, xrow, arow;
 };
 
-__device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, const FusedArgs& a) {
+__device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, const FusedArgs& a, int nmax) {
   FgUnit un;
   const int u1 = s.pref[n_exp] * a.mblk_gu;
   int v = u, nm = a.mblk_gu;
@@ -94,10 +104,19 @@ __device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, 
   while (e + 1 < n_exp && s.pref[e + 1] <= un.tile) ++e;
   const int nb = un.tile - s.pref[e];
   un.e = e;
-  un.nrows = min(kNMax, s.n[e] - nb * kNMax);
-  un.xrow = s.xrow[e] + nb * kNMax;
-  un.arow = s.arow[e] + nb * kNMax;
+  un.nrows = min(nmax, s.n[e] - nb * nmax);
+  un.xrow = s.xrow[e] + nb * nmax;
+  un.arow = s.arow[e] + nb * nmax;
   return un;
+}
+
+// Tiles of at most NMAX/2 tokens put two consecutive k-chunks of one weight
+// matrix in a stage (both 16 KB weight slots, 256 contiguous bytes per weight
+// row; the token slot holds both chunks' rows): down units stream W_down that
+// way; gate/up units alternate a gate stage and an up stage over the same two
+// k-chunks.
+__device__ __forceinline__ bool fg_paired(const FgUnit& un, const FusedArgs& a, int nmax) {
+  return un.nrows <= nmax / 2 && ((un.down ? a.kc_dn : a.kc_gu) & 1) == 0;
 }
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
@@ -109,18 +128,47 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Stages of a unit and the weight tiles of its stage j: (k offset, row) of the
+// first tile, the second tile (k offset, row) or k = -1 if the stage has one.
+struct FgStage {
+  int k0, row0, k1, row1;
+};
+__device__ __forceinline__ int fg_nstages(const FgUnit& un, const FusedArgs& a, bool pair) {
+  const int kcs = un.down ? a.kc_dn : a.kc_gu;
+  return pair ? (un.down ? kcs / 2 : kcs) : kcs;
+}
+__device__ __forceinline__ FgStage fg_stage(const FgUnit& un, const FusedArgs& a, bool pair, int j) {
+  FgStage g;
+  if (pair) {
+    const int kc = un.down ? 2 * j : 2 * (j >> 1);
+    const int row = (!un.down && (j & 1)) ? a.a_up_row + un.mb * kBM : un.mb * kBM;
+    g.k0 = kc * kBK;
+    g.row0 = row;
+    g.k1 = (kc + 1) * kBK;
+    g.row1 = row;
+  } else {
+    g.k0 = j * kBK;
+    g.row0 = un.mb * kBM;
+    g.k1 = un.down ? -1 : j * kBK;
+    g.row1 = a.a_up_row + un.mb * kBM;
+  }
+  return g;
+}
+
+template <int NMAX>
 __global__ void __launch_bounds__(192, 1)
     moe_expert_gemms(const __grid_constant__ CUtensorMap mGuR, const __grid_constant__ CUtensorMap mGuS,
                      const __grid_constant__ CUtensorMap mDnR, const __grid_constant__ CUtensorMap mDnS,
                      const __grid_constant__ CUtensorMap mXr, const __grid_constant__ CUtensorMap mXs,
                      const __grid_constant__ CUtensorMap mAct, const FusedArgs args) {
+  using C = FgCfg<NMAX>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
-  uint8_t* aux = smem + kFgStages * kFgStageBytes;
+  uint8_t* aux = smem + C::kStages * C::kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(aux);
-  uint64_t* empty = full + kFgStages;
-  uint64_t* tfull = empty + kFgStages;
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* ufull = tempty + 2;
   uint64_t* uempty = ufull + kFgRing;
@@ -134,7 +182,7 @@ __global__ void __launch_bounds__(192, 1)
   const int n_exp = args.E + args.S;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kFgStages; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -160,7 +208,7 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&mAct);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kFgTmemCols);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   if (warp == 2) {
@@ -183,7 +231,7 @@ __global__ void __launch_bounds__(192, 1)
       int acc = 0;
       for (int e = 0; e < n_exp; ++e) {
         sch->pref[e] = acc;
-        acc += cdiv(sch->n[e], kNMax);
+        acc += cdiv(sch->n[e], NMAX);
       }
       sch->pref[n_exp] = acc;
     }
@@ -209,14 +257,17 @@ __global__ void __launch_bounds__(192, 1)
       auto next_stage = [&]() {
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == kFgStages) {
+        if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1;
         }
       };
+      // the next ticket is requested one unit ahead so its round trip overlaps the loads
+      int next_u = atomicAdd(ticket, 1);
       while (true) {
-        int u = atomicAdd(ticket, 1);
+        int u = next_u;
         if (u >= total || *abort_flag) u = -1;
+        if (u >= 0) next_u = atomicAdd(ticket, 1);
         if (!mbar_wait(&uempty[slot], rphase ^ 1, limit)) {
           record_error(kErrTimeout, 130);
           *abort_flag = 1;
@@ -229,7 +280,7 @@ __global__ void __launch_bounds__(192, 1)
           rphase ^= 1;
         }
         if (u < 0) break;
-        const FgUnit un = fg_decode(u, *sch, n_exp, args);
+        const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
         const bool shared = un.e >= args.E;
         const int ecoord = shared ? un.e - args.E : un.e;
         const CUtensorMap* mA = un.down ? (shared ? &mDnS : &mDnR) : (shared ? &mGuS : &mGuR);
@@ -238,28 +289,38 @@ __global__ void __launch_bounds__(192, 1)
         const int brow0 = un.down ? un.arow : un.xrow;
         const int nbox = cdiv(un.nrows, box);
         const int kcs = un.down ? args.kc_dn : args.kc_gu;
-        const uint32_t bytes = (un.down ? 1 : 2) * kFgABytes + nbox * box * kBK * 2;
+        // a down tile of <= 64 tokens carries two consecutive k-chunks per stage
+        const bool pair = fg_paired(un, args, NMAX);
+        // stages of a unit: paired down: kcs/2; paired gate/up: kcs (gate, up, gate, ...); else kcs
+        const int nst = fg_nstages(un, args, pair);
+        const uint32_t bchunk = nbox * box * kBK * 2;
+        const uint32_t bytes = pair ? 2 * kFgABytes + 2 * bchunk : (un.down ? 1 : 2) * kFgABytes + bchunk;
         bool ok = true;
-        auto load_b = [&](int st, int kc) {
-          uint8_t* bt = tiles + st * kFgStageBytes + 2 * kFgABytes;
-          for (int j = 0; j < nbox; ++j)
-            tma_load_2d(bt + j * box * kBK * 2, mB, &full[st], kc * kBK, brow0 + j * box);
+        // first k-chunk of stage j
+        auto kc_of = [&](int j) { return pair ? (un.down ? 2 * j : 2 * (j >> 1)) : j; };
+        auto load_b = [&](int st, int j) {
+          uint8_t* bt = tiles + st * C::kStageBytes + 2 * kFgABytes;
+          for (int h = 0; h < (pair ? 2 : 1); ++h) {
+            const int kc = kc_of(j) + h;
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(bt + h * C::kPairBOff + b * box * kBK * 2, mB, &full[st], kc * kBK, brow0 + b * box);
+          }
         };
         // weights of the first stages go out before the activations are known to be ready
-        const int npre = un.down ? min(kFgStages, kcs) : 0;
+        const int npre = un.down ? min(C::kStages, nst) : 0;
         const int st0 = stage;
-        for (int kc = 0; kc < kcs && ok; ++kc) {
+        for (int kc = 0; kc < nst && ok; ++kc) {
           if (!mbar_wait(&empty[stage], phase ^ 1, limit)) {
             record_error(kErrTimeout, 131);
             *abort_flag = 1;
             ok = false;
             break;
           }
-          uint8_t* st = tiles + stage * kFgStageBytes;
+          uint8_t* st = tiles + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          const int kx = kc * kBK;
-          tma_load_3d_hint(st, mA, &full[stage], kx, un.mb * kBM, ecoord, pol_w);
-          if (!un.down) tma_load_3d_hint(st + kFgABytes, mA, &full[stage], kx, args.a_up_row + un.mb * kBM, ecoord, pol_w);
+          const FgStage g = fg_stage(un, args, pair, kc);
+          tma_load_3d_hint(st, mA, &full[stage], g.k0, g.row0, ecoord, pol_w);
+          if (g.k1 >= 0) tma_load_3d_hint(st + kFgABytes, mA, &full[stage], g.k1, g.row1, ecoord, pol_w);
           if (kc >= npre) load_b(stage, kc);
           if (kc + 1 == npre) {
             // every stage of the prefetch holds its weights in flight: now wait for the tile
@@ -273,14 +334,14 @@ __global__ void __launch_bounds__(192, 1)
               __nanosleep(64);
             }
             fence_proxy_async_global();
-            for (int j = 0; j < npre; ++j) load_b((st0 + j) % kFgStages, j);
+            for (int j = 0; j < npre; ++j) load_b((st0 + j) % C::kStages, j);
           }
           next_stage();
         }
         if (!ok) break;
       }
       // every issued copy has landed before the CTA may exit
-      for (int s = 0; s < kFgStages; ++s)
+      for (int s = 0; s < C::kStages; ++s)
         if (issued & (1u << s)) mbar_wait(&full[s], (last_par >> s) & 1, limit);
     }
   } else if (warp == 1) {
@@ -301,7 +362,7 @@ __global__ void __launch_bounds__(192, 1)
           rphase ^= 1;
         }
         if (u < 0 || *abort_flag) break;
-        const FgUnit un = fg_decode(u, *sch, n_exp, args);
+        const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
         const int ab = lu & 1;
         const uint32_t ap = (lu >> 1) & 1;
         ++lu;
@@ -312,11 +373,13 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_f32(kBM, cdiv(un.nrows, 16) * 16);
-        const uint32_t d0 = tmem_base + ab * kFgAccCols;
-        const uint32_t d1 = d0 + kNMax;
+        const uint32_t d0 = tmem_base + ab * C::kAccCols;
+        const uint32_t d1 = d0 + NMAX;
         const int kcs = un.down ? args.kc_dn : args.kc_gu;
+        const bool pair = fg_paired(un, args, NMAX);
+        const int nst = fg_nstages(un, args, pair);
         bool ok = true;
-        for (int kc = 0; kc < kcs; ++kc) {
+        for (int kc = 0; kc < nst; ++kc) {
           if (!mbar_wait(&full[stage], phase, limit)) {
             record_error(kErrTimeout, 135);
             *abort_flag = 1;
@@ -324,18 +387,29 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_u32(tiles + stage * kFgStageBytes);
+          const uint32_t st = smem_u32(tiles + stage * C::kStageBytes);
           const uint64_t a0 = sw128_kmajor_desc(st);
           const uint64_t a1 = sw128_kmajor_desc(st + kFgABytes);
           const uint64_t b = sw128_kmajor_desc(st + 2 * kFgABytes);
+          if (pair) {
+            // down: stage kc accumulates into d0; gate/up: even stages gate (d0), odd up (d1)
+            const uint64_t b1 = sw128_kmajor_desc(st + 2 * kFgABytes + C::kPairBOff);
+            const uint32_t d = (!un.down && (kc & 1)) ? d1 : d0;
+            const uint32_t first = un.down ? (kc == 0) : (kc < 2);
 #pragma unroll
-          for (int k16 = 0; k16 < kBK / 16; ++k16) {
-            const uint32_t acc = (kc | k16) != 0;
-            umma_bf16(d0, a0 + 2 * k16, b + 2 * k16, idesc, acc);
-            if (!un.down) umma_bf16(d1, a1 + 2 * k16, b + 2 * k16, idesc, acc);
+            for (int k16 = 0; k16 < kBK / 16; ++k16) umma_bf16(d, a0 + 2 * k16, b + 2 * k16, idesc, !(first && k16 == 0));
+#pragma unroll
+            for (int k16 = 0; k16 < kBK / 16; ++k16) umma_bf16(d, a1 + 2 * k16, b1 + 2 * k16, idesc, 1);
+          } else {
+#pragma unroll
+            for (int k16 = 0; k16 < kBK / 16; ++k16) {
+              const uint32_t acc = (kc | k16) != 0;
+              umma_bf16(d0, a0 + 2 * k16, b + 2 * k16, idesc, acc);
+              if (!un.down) umma_bf16(d1, a1 + 2 * k16, b + 2 * k16, idesc, acc);
+            }
           }
           umma_commit(&empty[stage]);
-          if (++stage == kFgStages) {
+          if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
           }
@@ -366,7 +440,7 @@ __global__ void __launch_bounds__(192, 1)
         rphase ^= 1;
       }
       if (u < 0 || *abort_flag) break;
-      const FgUnit un = fg_decode(u, *sch, n_exp, args);
+      const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
       const int ab = lu & 1;
       const uint32_t ap = (lu >> 1) & 1;
       ++lu;
@@ -376,13 +450,13 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + ab * kFgAccCols;
+      const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + ab * C::kAccCols;
       const int ld = un.down ? args.mblk_dn * kBM : args.mblk_gu * kBM;
       __nv_bfloat16* dst = (un.down ? args.out : args.act) + (size_t)un.arow * ld + un.mb * kBM + row;
       for (int c0 = 0; c0 < un.nrows; c0 += 16) {
         uint32_t g[16], v[16];
         tmem_ld16(t0 + c0, g);
-        if (!un.down) tmem_ld16(t0 + kNMax + c0, v);
+        if (!un.down) tmem_ld16(t0 + NMAX + c0, v);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -408,52 +482,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kFgTmemCols);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
-}
-
-// Weighted combine of the layer: out[t] = bf16(res + sum_s o_shared[s][t] +
-// sum_j g[t,j] * o[inv[t,j]]) with res = x[t] if add_residual else 0. One
-// thread per 8 consecutive hidden elements; fixed summation order.
-__global__ void __launch_bounds__(256) moe_combine(const __nv_bfloat16* __restrict__ x,
-                                                   const __nv_bfloat16* __restrict__ o,
-                                                   const int32_t* __restrict__ inv, const float* __restrict__ g,
-                                                   int T, int H, int k, int S, int add_residual,
-                                                   __nv_bfloat16* __restrict__ out) {
-  const int per_row = H / 8;
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= T * per_row) return;
-  const int t = i / per_row, c = i - t * per_row;
-  float y[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) y[j] = 0.0f;
-  for (int s = 0; s < S; ++s) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(o + ((size_t)k * T + (size_t)s * T + t) * H) + c);
-    y[0] += bf16_lo(v.x); y[1] += bf16_hi(v.x); y[2] += bf16_lo(v.y); y[3] += bf16_hi(v.y);
-    y[4] += bf16_lo(v.z); y[5] += bf16_hi(v.z); y[6] += bf16_lo(v.w); y[7] += bf16_hi(v.w);
-  }
-  for (int j = 0; j < k; ++j) {
-    const int p = inv[t * k + j];
-    const float gj = g[t * k + j];
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(o + (size_t)p * H) + c);
-    y[0] = __fmaf_rn(gj, bf16_lo(v.x), y[0]); y[1] = __fmaf_rn(gj, bf16_hi(v.x), y[1]);
-    y[2] = __fmaf_rn(gj, bf16_lo(v.y), y[2]); y[3] = __fmaf_rn(gj, bf16_hi(v.y), y[3]);
-    y[4] = __fmaf_rn(gj, bf16_lo(v.z), y[4]); y[5] = __fmaf_rn(gj, bf16_hi(v.z), y[5]);
-    y[6] = __fmaf_rn(gj, bf16_lo(v.w), y[6]); y[7] = __fmaf_rn(gj, bf16_hi(v.w), y[7]);
-  }
-  if (add_residual) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H) + c);
-    y[0] += bf16_lo(v.x); y[1] += bf16_hi(v.x); y[2] += bf16_lo(v.y); y[3] += bf16_hi(v.y);
-    y[4] += bf16_lo(v.z); y[5] += bf16_hi(v.z); y[6] += bf16_lo(v.w); y[7] += bf16_hi(v.w);
-  }
-  uint4 r;
-  __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
-  __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]), h3 = __floats2bfloat162_rn(y[6], y[7]);
-  r.x = *reinterpret_cast<uint32_t*>(&h0);
-  r.y = *reinterpret_cast<uint32_t*>(&h1);
-  r.z = *reinterpret_cast<uint32_t*>(&h2);
-  r.w = *reinterpret_cast<uint32_t*>(&h3);
-  reinterpret_cast<uint4*>(out + (size_t)t * H)[c] = r;
 }
 
 }  // namespace vg

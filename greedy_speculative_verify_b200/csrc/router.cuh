@@ -3,10 +3,12 @@
 // Top-6 of 64 routed experts per token ("Jina AI's 3.4B OCR model targets faster
 // page parsing", "A compressed visual front end"; jina-ocr-v1 model card,
 // architecture paragraph). The pages give no formula. Reading used here:
-//  * l[t,e] = fp32 fused-multiply-add chain over h = 0..H-1 starting at +0,
-//    then + bias[e] in one fp32 addition. The order is part of the definition
-//    so that the selected experts are reproducible bit for bit; both kernels
-//    below keep each output's chain in one thread, in increasing h.
+//  * l[t,e] = sum_h x[t,h] w[e,h] in fp32 as four partial sums over the
+//    contiguous quarters of h, each an fma chain in increasing h from +0,
+//    combined as (q0 + q1) + (q2 + q3), then + bias[e] in one fp32 addition.
+//    The order is part of the definition so that the selected experts are
+//    reproducible bit for bit; the quarter chains keep the critical path at
+//    H/4 dependent fmas.
 //  * selection by (l descending, e ascending); softmax over all E logits,
 //    weights not renormalised over the selected experts.
 #pragma once
@@ -77,76 +79,11 @@ __device__ __forceinline__ void topk_softmax_warp(const float* l, int lane, int3
   }
 }
 
-// Small token counts: one thread per (token, expert) output, 4 tokens x 64
-// experts per block. The router weights and the 4 token rows stream through
-// shared memory in 128-element chunks with cp.async double buffering, so the
-// only latency left on the critical path is the fma chain itself.
-constexpr int kRtChunk = 128;               // k per chunk
-constexpr int kRtWStride = kRtChunk + 8;    // padded row (272 B): conflict-free 16-byte reads
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-template <int K>
-__global__ void __launch_bounds__(256) router_topk_small(const __nv_bfloat16* __restrict__ x,
-                                                         const __nv_bfloat16* __restrict__ w,
-                                                         const float* __restrict__ bias, int T, int H,
-                                                         int32_t* __restrict__ idx_out,
-                                                         float* __restrict__ w_out) {
-  __shared__ __align__(16) __nv_bfloat16 ws[2][kRouterE * kRtWStride];
-  __shared__ __align__(16) __nv_bfloat16 xs[2][4 * kRtChunk];
-  __shared__ float logit[4][kRouterE];
-  const int tid = threadIdx.x;
-  const int tl = tid >> 6, e = tid & 63;
-  const int t0 = blockIdx.x * 4;
-  const int nchunks = H / kRtChunk;
-
-  auto load_chunk = [&](int c, int buf) {
-    const int k0 = c * kRtChunk;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {  // 64 rows x 16 pieces of 16 B
-      const int q = tid + i * 256;
-      const int row = q >> 4, piece = q & 15;
-      cp_async16(&ws[buf][row * kRtWStride + piece * 8], w + (size_t)row * H + k0 + piece * 8);
-    }
-    if (tid < 64) {  // 4 token rows x 16 pieces
-      const int row = tid >> 4, piece = tid & 15;
-      const int t = min(t0 + row, T - 1);
-      cp_async16(&xs[buf][row * kRtChunk + piece * 8], x + (size_t)t * H + k0 + piece * 8);
-    }
-    cp_async_commit();
-  };
-
-  float acc = 0.0f;
-  load_chunk(0, 0);
-  for (int c = 0; c < nchunks; ++c) {
-    const int buf = c & 1;
-    if (c + 1 < nchunks) {
-      load_chunk(c + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint4* wr = reinterpret_cast<const uint4*>(&ws[buf][e * kRtWStride]);
-    const uint4* xr = reinterpret_cast<const uint4*>(&xs[buf][tl * kRtChunk]);
-#pragma unroll
-    for (int p = 0; p < kRtChunk / 8; ++p) fma8(acc, xr[p], wr[p]);
-    __syncthreads();
-  }
-  if (bias != nullptr) acc = __fadd_rn(acc, bias[e]);
-  logit[tl][e] = acc;
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  if (warp < 4) {
-    const int tt = t0 + warp;
-    if (tt < T) topk_softmax_warp<K>(logit[warp], lane, idx_out + (size_t)tt * K, w_out + (size_t)tt * K);
-  }
-}
+// Decode sizes compute the logits inside the layer-entry kernel
+// (layer_entry.cuh): 16-expert slices of the router weights in shared memory as
+// padded quarter rows, four threads per (token, expert) output.
+constexpr int kRtExperts = 16;  // experts per router slice
+constexpr int kRtPad = 8;       // elements of padding per quarter row: conflict-free 16-byte reads
 
 // Large token counts: a 128-token x 64-expert block tile, staged through shared
 // memory 32 k at a time; each thread owns 8 tokens x 4 experts and runs every
@@ -164,11 +101,14 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
   const int tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;
   const int t0 = blockIdx.x * BT;
-  float acc[8][4];
+  // quarter sums: acc runs the current quarter's chains; q01 and q2 keep the
+  // finished ones until (q0 + q1) + (q2 + q3) (H/4 is a multiple of BK)
+  float acc[8][4], q01[8][4], q2[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = q01[i][j] = q2[i][j] = 0.0f;
+  const int HQ = H / 4;
 
   for (int k0 = 0; k0 < H; k0 += BK) {
     // x tile: 128 tokens x 32 k = 512 uint4
@@ -213,6 +153,19 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
         for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(av[i], bv[j], acc[i][j]);
     }
     __syncthreads();
+    const int qend = (k0 + BK) / HQ;  // a quarter ends with this chunk when (k0 + BK) % HQ == 0
+    if ((k0 + BK) % HQ == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (qend == 1) q01[i][j] = acc[i][j];
+          else if (qend == 2) q01[i][j] = q01[i][j] + acc[i][j];
+          else if (qend == 3) q2[i][j] = acc[i][j];
+          else q01[i][j] = q01[i][j] + (q2[i][j] + acc[i][j]);
+          acc[i][j] = 0.0f;
+        }
+    }
   }
   float* logits = buf;
 #pragma unroll
@@ -221,7 +174,7 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
     const float b = bias != nullptr ? bias[e] : 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float v = acc[i][j];
+      float v = q01[i][j];
       if (bias != nullptr) v = __fadd_rn(v, b);
       logits[(ty * 8 + i) * LS + e] = v;
     }

@@ -14,7 +14,7 @@ namespace vg {
 
 constexpr int kSortE = 64;
 constexpr int kSortChunk = 1024;       // assignments per pass (one per thread)
-constexpr int kSortSmallMax = 8192;    // single-kernel path up to this many assignments
+constexpr int kSortSmallMax = 8192;    // decode path (layer-entry kernel) up to this many assignments
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -22,9 +22,10 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-// Positions of the 1024 assignments a = base + threadIdx.x given the running
-// start of every expert's segment `run` (shared). Returns -1 for a >= N.
-// Advances `run` by this chunk's counts. Must be called by all 1024 threads.
+// Positions of the blockDim.x assignments a = base + threadIdx.x given the
+// running start of every expert's segment `run` (shared). Returns -1 for a >= N.
+// Advances `run` by this chunk's counts. Must be called by every thread of the
+// block (at most 1024).
 __device__ __forceinline__ int chunk_positions(const int32_t* __restrict__ keys, int base, int N, int* run,
                                                int (*wcnt)[kSortE]) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -79,53 +80,6 @@ __device__ __forceinline__ void gather_rows(const __nv_bfloat16* __restrict__ x,
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)token * H);
   uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * H);
   for (int c = threadIdx.x & 31; c < H / 8; c += 32) dst[c] = __ldg(src + c);
-}
-
-// Single-kernel path (N <= kSortSmallMax). Every block computes the whole
-// (deterministic) sort in shared memory; block 0 writes offsets/perm/inv; every
-// block gathers the rows at positions blockIdx.x, blockIdx.x + gridDim.x, ...
-__global__ void __launch_bounds__(1024) expert_sort_small(const int32_t* __restrict__ keys, int N, int k,
-                                                          int32_t* __restrict__ offsets,
-                                                          int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                                          const __nv_bfloat16* __restrict__ x, int H,
-                                                          __nv_bfloat16* __restrict__ x_perm,
-                                                          int32_t* __restrict__ sched, int sched_len) {
-  extern __shared__ int32_t perm_s[];  // [N]
-  __shared__ int cnt[kSortE], run[kSortE];
-  __shared__ int wcnt[32][kSortE];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid < kSortE) cnt[tid] = 0;
-  if (blockIdx.x == 0)  // the expert GEMMs' ticket counter and per-tile readiness words
-    for (int i = tid; i < sched_len; i += blockDim.x) sched[i] = 0;
-  __syncthreads();
-  for (int a = tid; a < N; a += blockDim.x) {
-    const int key = keys[a];
-    if ((unsigned)key < (unsigned)kSortE) atomicAdd(&cnt[key], 1);
-  }
-  __syncthreads();
-  if (warp == 0) {
-    scan64_warp(cnt, run, lane);
-    if (blockIdx.x == 0) {
-      offsets[2 * lane] = run[2 * lane];
-      offsets[2 * lane + 1] = run[2 * lane + 1];
-      if (lane == 0) offsets[kSortE] = N;
-    }
-  }
-  __syncthreads();
-  for (int base = 0; base < N; base += kSortChunk) {
-    const int pos = chunk_positions(keys, base, N, run, wcnt);
-    const int a = base + tid;
-    if (pos >= 0) {
-      perm_s[pos] = a;
-      if (blockIdx.x == 0) {
-        perm[pos] = a;
-        inv[a] = pos;
-      }
-    }
-  }
-  __syncthreads();
-  for (int row = blockIdx.x + warp * gridDim.x; row < N; row += 32 * gridDim.x)
-    gather_rows(x, x_perm, H, row, perm_s[row] / k);
 }
 
 // Multi-kernel path, pass 1: per-chunk histograms [nchunks][64].

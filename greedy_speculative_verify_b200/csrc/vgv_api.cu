@@ -9,7 +9,9 @@
 
 #include "vgv.h"
 #include "common.cuh"
+#include "combine.cuh"
 #include "gemm_moe.cuh"
+#include "layer_entry.cuh"
 #include "lmhead.cuh"
 #include "router.cuh"
 #include "sort.cuh"
@@ -18,7 +20,6 @@ namespace {
 
 constexpr int kH = 1280, kI = 896, kE = 64, kS = 2, kTopK = 6;
 constexpr int kMaxDevices = 64;
-constexpr int kSmallRouterMaxT = 512;
 
 struct DevState {
   bool init = false;
@@ -37,6 +38,16 @@ ProfHook g_prof[VG_KERNEL_KINDS];
 std::mutex g_prof_mu;
 bool g_prof_any = false;
 
+// Records an event on `s`; while `s` is being captured into a graph the record
+// must be marked external to become a timing node of the graph.
+void record_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, s);
+}
+
 // Brackets one launch of `kind` with the hook's events, if any are set.
 struct ProfScope {
   int kind;
@@ -48,13 +59,13 @@ struct ProfScope {
     ProfHook& h = g_prof[kind];
     if (h.starts.empty()) return;
     slot = h.count++ % (int64_t)h.starts.size();
-    cudaEventRecord(h.starts[slot], s);
+    record_event(h.starts[slot], s);
   }
   ~ProfScope() {
     if (slot < 0) return;
     std::lock_guard<std::mutex> lk(g_prof_mu);
     ProfHook& h = g_prof[kind];
-    if ((int64_t)h.stops.size() > slot) cudaEventRecord(h.stops[slot], s);
+    if ((int64_t)h.stops.size() > slot) record_event(h.stops[slot], s);
   }
 };
 
@@ -71,14 +82,16 @@ vg_status device_state(DevState** out) {
   DevState& d = g_dev[dev];
   if (!d.init) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cuda_fail();
-    if (cudaFuncSetAttribute(vg::moe_expert_gemms, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::kFgSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(vg::moe_expert_gemms<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::FgCfg<128>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vg::moe_expert_gemms<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::FgCfg<64>::kSmemBytes) != cudaSuccess)
+      return cuda_fail();
+    if (cudaFuncSetAttribute(vg::moe_layer_entry<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::layer_entry_smem(kH, vg::kSortSmallMax)) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
-      return cuda_fail();
-    if (cudaFuncSetAttribute(vg::expert_sort_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::kSortSmallMax * 4) != cudaSuccess)
       return cuda_fail();
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
@@ -117,13 +130,17 @@ bool dims_supported(const vg_moe_dims* d) {
 }
 
 struct MoeWs {
-  size_t idx, w, offsets, perm, inv, xperm, act, o, ccnt, cbase, sched, total;
+  size_t idx, w, logits, offsets, perm, inv, xperm, act, o, ccnt, cbase, sched, gbar, total;
   int sched_len;
 };
 
 // Upper bound of the expert GEMMs' token tiles: routed segments cut at 128 plus
 // one partial tile per routed expert, plus the shared experts' tiles.
-int max_tiles(int T) { return vg::cdiv(T * kTopK, vg::kNMax) + kE + kS * vg::cdiv(T, vg::kNMax); }
+int max_tiles(int T) { return vg::cdiv(T * kTopK, 64) + kE + kS * vg::cdiv(T, 64); }
+
+// Tile width of the expert GEMMs: 64-token tiles (and a fifth pipeline stage)
+// at decode sizes, 128-token tiles for prefill-sized segments.
+int expert_tile(int T) { return T <= 1024 ? 64 : 128; }
 
 MoeWs moe_layout(int T) {
   const size_t N = (size_t)T * kTopK;
@@ -137,6 +154,7 @@ MoeWs moe_layout(int T) {
   };
   L.idx = take(N * 4);
   L.w = take(N * 4);
+  L.logits = take((size_t)T * kE * 4);
   L.offsets = take((kE + 1) * 4);
   L.perm = take(N * 4);
   L.inv = take(N * 4);
@@ -147,6 +165,7 @@ MoeWs moe_layout(int T) {
   L.cbase = take(nch * kE * 4);
   L.sched_len = 1 + max_tiles(T);
   L.sched = take((size_t)L.sched_len * 4);
+  L.gbar = take(8);
   L.total = off;
   return L;
 }
@@ -156,103 +175,192 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-// Launches one MoE layer; arguments already validated.
-vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, const float* router_bias,
-                     const void* expert_w, const void* shared_w, int add_residual, void* out,
-                     const vg_moe_taps* taps, void* workspace, cudaStream_t s) {
-  using namespace vg;
+// Device buffers of one layer inside the workspace (or the caller's taps).
+struct LayerBufs {
+  int32_t *idx, *offsets, *perm, *inv, *sched, *ccnt, *cbase;
+  float *gw, *logits;
+  uint32_t* gbar;
+  __nv_bfloat16 *xperm, *act, *o;
+  int sched_len;
+};
+
+LayerBufs carve(void* workspace, int T, const vg_moe_taps* taps) {
   const MoeWs L = moe_layout(T);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int32_t* idx = (taps && taps->topk_idx) ? taps->topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
-  float* gw = (taps && taps->topk_weight) ? taps->topk_weight : reinterpret_cast<float*>(ws + L.w);
-  int32_t* offsets = (taps && taps->expert_offsets) ? taps->expert_offsets : reinterpret_cast<int32_t*>(ws + L.offsets);
-  int32_t* perm = (taps && taps->perm) ? taps->perm : reinterpret_cast<int32_t*>(ws + L.perm);
-  int32_t* inv = (taps && taps->inv_perm) ? taps->inv_perm : reinterpret_cast<int32_t*>(ws + L.inv);
-  __nv_bfloat16* xperm = reinterpret_cast<__nv_bfloat16*>(ws + L.xperm);
-  __nv_bfloat16* act = (taps && taps->act) ? static_cast<__nv_bfloat16*>(taps->act) : reinterpret_cast<__nv_bfloat16*>(ws + L.act);
-  __nv_bfloat16* o = (taps && taps->expert_out) ? static_cast<__nv_bfloat16*>(taps->expert_out) : reinterpret_cast<__nv_bfloat16*>(ws + L.o);
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  LayerBufs b{};
+  b.idx = (taps && taps->topk_idx) ? taps->topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
+  b.gw = (taps && taps->topk_weight) ? taps->topk_weight : reinterpret_cast<float*>(ws + L.w);
+  b.offsets = (taps && taps->expert_offsets) ? taps->expert_offsets : reinterpret_cast<int32_t*>(ws + L.offsets);
+  b.perm = (taps && taps->perm) ? taps->perm : reinterpret_cast<int32_t*>(ws + L.perm);
+  b.inv = (taps && taps->inv_perm) ? taps->inv_perm : reinterpret_cast<int32_t*>(ws + L.inv);
+  b.act = (taps && taps->act) ? static_cast<__nv_bfloat16*>(taps->act) : reinterpret_cast<__nv_bfloat16*>(ws + L.act);
+  b.o = (taps && taps->expert_out) ? static_cast<__nv_bfloat16*>(taps->expert_out)
+                                   : reinterpret_cast<__nv_bfloat16*>(ws + L.o);
+  b.logits = reinterpret_cast<float*>(ws + L.logits);
+  b.xperm = reinterpret_cast<__nv_bfloat16*>(ws + L.xperm);
+  b.sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  b.sched_len = L.sched_len;
+  b.ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
+  b.cbase = reinterpret_cast<int32_t*>(ws + L.cbase);
+  b.gbar = reinterpret_cast<uint32_t*>(ws + L.gbar);
+  return b;
+}
+
+bool small_path(int T) { return (int64_t)T * kTopK <= vg::kSortSmallMax; }
+
+// The previous layer's combine, when it is folded into this layer's entry.
+struct PrevCombine {
+  const __nv_bfloat16* x;  // previous layer's input (residual)
+  const LayerBufs* b;      // previous layer's buffers (o, inv, gw)
+};
+
+// Router, top-k and grouping of a layer whose input is xcur (computed first from
+// `prev` when given: decode path only). Large token counts: separate kernels.
+// `nbar` counts the grid barriers passed on b.gbar since it was zeroed (host side:
+// every launch passes the same number, so it is known without reading the device).
+vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv_bfloat16* x_in,
+                       __nv_bfloat16* x_out, const void* router_w, const float* router_bias, const LayerBufs& b,
+                       uint32_t* nbar, cudaStream_t s) {
+  using namespace vg;
   const int N = T * kTopK;
-  int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
-
-  // 1. router
-  {
-  ProfScope ps(VG_KERNEL_ROUTER, s);
-  if (T <= kSmallRouterMaxT)
-    router_topk_small<kTopK><<<cdiv(T, 4), 256, 0, s>>>(xb, static_cast<const __nv_bfloat16*>(router_w),
-                                                       router_bias, T, kH, idx, gw);
-  else
-    router_topk_tiled<kTopK><<<cdiv(T, 128), 256, 0, s>>>(xb, static_cast<const __nv_bfloat16*>(router_w),
-                                                         router_bias, T, kH, idx, gw);
-  }
-  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
-
-  // 2. grouping by expert + row gather
-  {
-  ProfScope ps(VG_KERNEL_GROUPING, s);
-  if (N <= kSortSmallMax) {
-    const int grid = min(dev->sms, N);
-    expert_sort_small<<<grid, 1024, N * 4, s>>>(idx, N, kTopK, offsets, perm, inv, xb, kH, xperm, sched,
-                                                L.sched_len);
-  } else {
-    const int nch = cdiv(N, kSortChunk);
-    int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
-    int32_t* cbase = reinterpret_cast<int32_t*>(ws + L.cbase);
-    expert_hist_chunks<<<nch, 1024, 0, s>>>(idx, N, ccnt);
-    expert_scan_chunks<<<1, 64, 0, s>>>(ccnt, nch, N, offsets, cbase, sched, L.sched_len);
-    expert_scatter_chunks<<<nch, 1024, 0, s>>>(idx, N, kTopK, cbase, perm, inv, xb, kH, xperm);
-  }
-  }
-  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
-
-  // 3. expert GEMMs: gate/up + SwiGLU then down, routed and shared experts, one launch
-  {
-    const uint64_t estride = (uint64_t)3 * kI * kH * 2;
-    const __nv_bfloat16* dr = static_cast<const __nv_bfloat16*>(expert_w) + (size_t)2 * kI * kH;
-    const __nv_bfloat16* dsh = static_cast<const __nv_bfloat16*>(shared_w) + (size_t)2 * kI * kH;
-    CUtensorMap mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct;
-    const uint64_t dGu[3] = {kH, 2 * kI, kE}, dGuS[3] = {kH, 2 * kI, kS}, sGu[2] = {kH * 2, estride};
-    const uint64_t dDn[3] = {kI, kH, kE}, dDnS[3] = {kI, kH, kS}, sDn[2] = {kI * 2, estride};
-    const uint32_t bA[3] = {kBK, kBM, 1};
-    const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
-    const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
-    const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
-    const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
-    const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, kBoxRows)};
-    if (make_map(&mGuR, expert_w, 3, dGu, sGu, bA) || make_map(&mGuS, shared_w, 3, dGuS, sGu, bA) ||
-        make_map(&mDnR, dr, 3, dDn, sDn, bA) || make_map(&mDnS, dsh, 3, dDnS, sDn, bA) ||
-        make_map(&mXr, xperm, 2, dXr, sX, bXr) || make_map(&mXs, x, 2, dXs, sX, bXs) ||
-        make_map(&mAct, act, 2, dAct, sAct, bAct))
-      return VG_ERR_CUDA;
-    FusedArgs a{};
-    a.offsets = offsets;
+  if (small_path(T)) {
+    EntryArgs a{};
+    if (prev) {
+      a.prev_o = prev->b->o;
+      a.prev_inv = prev->b->inv;
+      a.prev_gate = prev->b->gw;
+      a.prev_x = prev->x;
+      a.prev_add_residual = 1;
+      a.x_out = x_out;
+    }
+    a.x_in = x_in;
+    a.w = static_cast<const __nv_bfloat16*>(router_w);
+    a.bias = router_bias;
     a.T = T;
-    a.E = kE;
+    a.H = kH;
+    a.k = kTopK;
     a.S = kS;
-    a.mblk_gu = kI / kBM;
-    a.mblk_dn = kH / kBM;
-    a.kc_gu = kH / kBK;
-    a.kc_dn = kI / kBK;
-    a.a_up_row = kI;
-    a.box_xr = (int)bXr[1];
-    a.box_xs = (int)bXs[1];
-    a.box_act = (int)bAct[1];
-    a.sched = sched;
-    a.act = act;
-    a.out = o;
-    const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
-    ProfScope ps(VG_KERNEL_EXPERTS, s);
-    moe_expert_gemms<<<grid, 192, kFgSmemBytes, s>>>(mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct, a);
-    if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+    a.logits = b.logits;
+    a.idx = b.idx;
+    a.gate = b.gw;
+    a.offsets = b.offsets;
+    a.perm = b.perm;
+    a.inv = b.inv;
+    a.x_perm = b.xperm;
+    a.sched = b.sched;
+    a.sched_len = b.sched_len;
+    a.gbar = b.gbar;
+    a.gbar_base = *nbar;
+    const int grid = min(dev->sms, cdiv(T, kEntryTok));
+    if (grid > 1) *nbar += prev ? 2 : 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kEntryThreads);
+    cfg.dynamicSmemBytes = layer_entry_smem(kH, N);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    CUtensorMap mR;
+    const uint64_t dR[2] = {kH, kE}, sR[1] = {kH * 2};
+    const uint32_t bR[2] = {64, kE};
+    if (make_map(&mR, router_w, 2, dR, sR, bR)) return VG_ERR_CUDA;
+    ProfScope ps(VG_KERNEL_ROUTER, s);
+    if (cudaLaunchKernelEx(&cfg, moe_layer_entry<kTopK>, mR, a) != cudaSuccess) return cuda_fail();
+    return VG_OK;
   }
-  // 5. weighted combine + residual
+  const __nv_bfloat16* xcur = x_in;
+  if (prev) {
+    moe_combine<<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(prev->x, prev->b->o, prev->b->inv, prev->b->gw, T, kH,
+                                                       kTopK, kS, 1, x_out);
+    xcur = x_out;
+  }
   {
-    ProfScope ps(VG_KERNEL_COMBINE, s);
-    moe_combine<<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(xb, o, inv, gw, T, kH, kTopK, kS, add_residual,
-                                                       static_cast<__nv_bfloat16*>(out));
+    ProfScope ps(VG_KERNEL_ROUTER, s);
+    router_topk_tiled<kTopK><<<cdiv(T, 128), 256, 0, s>>>(xcur, static_cast<const __nv_bfloat16*>(router_w),
+                                                         router_bias, T, kH, b.idx, b.gw);
+  }
+  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  {
+    ProfScope ps(VG_KERNEL_GROUPING, s);
+    const int nch = cdiv(N, kSortChunk);
+    expert_hist_chunks<<<nch, 1024, 0, s>>>(b.idx, N, b.ccnt);
+    expert_scan_chunks<<<1, 64, 0, s>>>(b.ccnt, nch, N, b.offsets, b.cbase, b.sched, b.sched_len);
+    expert_scatter_chunks<<<nch, 1024, 0, s>>>(b.idx, N, kTopK, b.cbase, b.perm, b.inv, xcur, kH, b.xperm);
   }
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   return VG_OK;
+}
+
+// Expert GEMMs (gate/up + SwiGLU, down) of a layer with input x.
+vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert_w, const void* shared_w,
+                         const LayerBufs& b, cudaStream_t s) {
+  using namespace vg;
+  const int N = T * kTopK;
+  const uint64_t estride = (uint64_t)3 * kI * kH * 2;
+  const __nv_bfloat16* dr = static_cast<const __nv_bfloat16*>(expert_w) + (size_t)2 * kI * kH;
+  const __nv_bfloat16* dsh = static_cast<const __nv_bfloat16*>(shared_w) + (size_t)2 * kI * kH;
+  CUtensorMap mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct;
+  const uint64_t dGu[3] = {kH, 2 * kI, kE}, dGuS[3] = {kH, 2 * kI, kS}, sGu[2] = {kH * 2, estride};
+  const uint64_t dDn[3] = {kI, kH, kE}, dDnS[3] = {kI, kH, kS}, sDn[2] = {kI * 2, estride};
+  const uint32_t bA[3] = {kBK, kBM, 1};
+  const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
+  const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
+  const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
+  const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
+  const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, kBoxRows)};
+  if (make_map(&mGuR, expert_w, 3, dGu, sGu, bA) || make_map(&mGuS, shared_w, 3, dGuS, sGu, bA) ||
+      make_map(&mDnR, dr, 3, dDn, sDn, bA) || make_map(&mDnS, dsh, 3, dDnS, sDn, bA) ||
+      make_map(&mXr, b.xperm, 2, dXr, sX, bXr) || make_map(&mXs, x, 2, dXs, sX, bXs) ||
+      make_map(&mAct, b.act, 2, dAct, sAct, bAct))
+    return VG_ERR_CUDA;
+  FusedArgs a{};
+  a.offsets = b.offsets;
+  a.T = T;
+  a.E = kE;
+  a.S = kS;
+  a.mblk_gu = kI / kBM;
+  a.mblk_dn = kH / kBM;
+  a.kc_gu = kH / kBK;
+  a.kc_dn = kI / kBK;
+  a.a_up_row = kI;
+  a.box_xr = (int)bXr[1];
+  a.box_xs = (int)bXs[1];
+  a.box_act = (int)bAct[1];
+  a.sched = b.sched;
+  a.act = b.act;
+  a.out = b.o;
+  const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
+  ProfScope ps(VG_KERNEL_EXPERTS, s);
+  if (expert_tile(T) == 64)
+    moe_expert_gemms<64><<<grid, 192, FgCfg<64>::kSmemBytes, s>>>(mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct, a);
+  else
+    moe_expert_gemms<128><<<grid, 192, FgCfg<128>::kSmemBytes, s>>>(mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct, a);
+  return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+vg_status launch_combine(int T, const void* x, const LayerBufs& b, int add_residual, void* out, cudaStream_t s) {
+  using namespace vg;
+  ProfScope ps(VG_KERNEL_COMBINE, s);
+  moe_combine<<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), b.o, b.inv, b.gw, T, kH,
+                                                     kTopK, kS, add_residual, static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+// One layer: entry, expert GEMMs, combine into out.
+vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, const float* router_bias,
+                     const void* expert_w, const void* shared_w, int add_residual, void* out,
+                     const vg_moe_taps* taps, void* workspace, cudaStream_t s) {
+  const LayerBufs b = carve(workspace, T, taps);
+  if (cudaMemsetAsync(b.gbar, 0, 8, s) != cudaSuccess) return cuda_fail();
+  uint32_t nbar = 0;
+  vg_status st = launch_entry(dev, T, nullptr, static_cast<const __nv_bfloat16*>(x), nullptr, router_w, router_bias,
+                              b, &nbar, s);
+  if (st == VG_OK) st = launch_experts(dev, T, x, expert_w, shared_w, b, s);
+  if (st == VG_OK) st = launch_combine(T, x, b, add_residual, out, s);
+  return st;
 }
 
 size_t verify_ws_bytes(int B, int K, int V) {
@@ -340,15 +448,30 @@ vg_status vg_moe_ffn_stack(const vg_moe_dims* dims, int32_t n_layers, int32_t T,
   DevState* dev = nullptr;
   if ((st = device_state(&dev)) != VG_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* buf[2] = {ws + mw, ws + mw + hb};
-  const void* cur = x;
+  __nv_bfloat16* buf[2] = {reinterpret_cast<__nv_bfloat16*>(ws + mw), reinterpret_cast<__nv_bfloat16*>(ws + mw + hb)};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // x_0 = x; x_l (l >= 1) = buf[(l-1) & 1] is computed by layer l's entry from
+  // layer l-1's expert outputs; the last layer's combine writes out.
+  const LayerBufs b = carve(workspace, T, nullptr);
+  if (cudaMemsetAsync(b.gbar, 0, 8, s) != cudaSuccess) return cuda_fail();
+  uint32_t nbar = 0;
+  const __nv_bfloat16* xin = static_cast<const __nv_bfloat16*>(x);
   for (int l = 0; l < n_layers; ++l) {
-    void* dst = (l == n_layers - 1) ? out : buf[l & 1];
-    st = launch_moe(dev, T, cur, router_w[l], router_bias ? router_bias[l] : nullptr, expert_w[l], shared_w[l], 1,
-                    dst, nullptr, workspace, reinterpret_cast<cudaStream_t>(stream));
+    const __nv_bfloat16* xl = xin;
+    PrevCombine prev{xin, &b};
+    __nv_bfloat16* xout = nullptr;
+    if (l > 0) {
+      xout = buf[(l - 1) & 1];
+      xl = xout;
+    }
+    st = launch_entry(dev, T, l > 0 ? &prev : nullptr, xin, xout, router_w[l], router_bias ? router_bias[l] : nullptr,
+                      b, &nbar, s);
+    if (st == VG_OK) st = launch_experts(dev, T, xl, expert_w[l], shared_w[l], b, s);
     if (st != VG_OK) return st;
-    cur = dst;
+    xin = xl;
   }
+  st = launch_combine(T, xin, b, 1, out, s);
+  if (st != VG_OK) return st;
   return VG_OK;
 }
 

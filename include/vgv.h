@@ -169,10 +169,12 @@ vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V,
 
 /* Kernel kinds for the timing hook. */
 typedef enum vg_kernel {
-  VG_KERNEL_ROUTER = 0,    /* router logits + top-k + softmax */
-  VG_KERNEL_GROUPING = 1,  /* histogram, stable permutation, row gather */
+  VG_KERNEL_ROUTER = 0,    /* router + top-k (+ grouping, and the previous layer's
+                              combine inside a layer stack, at decode sizes) */
+  VG_KERNEL_GROUPING = 1,  /* histogram, stable permutation, row gather (large T) */
   VG_KERNEL_EXPERTS = 2,   /* expert GEMMs: gate/up + SwiGLU, then down (one launch) */
-  VG_KERNEL_COMBINE = 3,   /* weighted combine + shared experts + residual */
+  VG_KERNEL_COMBINE = 3,   /* weighted combine + shared experts + residual (a
+                              layer's own output, or the stack's last layer) */
   VG_KERNEL_LM_HEAD = 4,   /* LM-head GEMM + per-tile argmax */
   VG_KERNEL_ACCEPT = 5,    /* argmax reduction + prefix accept */
   VG_KERNEL_KINDS = 6

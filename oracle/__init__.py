@@ -24,8 +24,9 @@ What the pages fix, and where each piece comes from:
 
 Readings where the pages are silent (each one is listed in the design doc):
 
-* router logits are an fp32 fused-multiply-add chain over h = 0..H-1 starting
-  at +0, then + b_e in fp32; selection is on the logits (descending, ties to the
+* router logits are four fp32 fused-multiply-add chains over the contiguous
+  quarters of h (each from +0, increasing h), combined as (q0+q1)+(q2+q3) in
+  fp32, then + b_e in fp32; selection is on the logits (descending, ties to the
   lower expert index); gate weights are the softmax over all E logits with no
   renormalisation over the selected six;
 * expert FFN = SwiGLU: down(silu(gate x) * up x), silu(z) = z / (1 + e^-z);
@@ -39,14 +40,14 @@ Readings where the pages are silent (each one is listed in the design doc):
 Every function is dimension-generic so the self-tests can run on tiny shapes.
 """
 from .bf16 import widen, round_bf16_bits
-from .router import router_logits, route, softmax_gates
+from .router import router_logits, route, softmax_gates, segment_bounds
 from .permute import expert_permutation
 from .experts import silu, swiglu_expert, moe_ffn, moe_stack
 from .verify import lm_head_argmax, logit_fp64, prefix_accept, tau, acceptance_rate
 from .decode import MarkovDecoder, greedy_decode, speculative_decode
 
 __all__ = [
-    "widen", "round_bf16_bits", "router_logits", "route", "softmax_gates",
+    "widen", "round_bf16_bits", "router_logits", "route", "softmax_gates", "segment_bounds",
     "expert_permutation", "silu", "swiglu_expert", "moe_ffn", "moe_stack",
     "lm_head_argmax", "logit_fp64", "prefix_accept", "tau", "acceptance_rate",
     "MarkovDecoder", "greedy_decode", "speculative_decode",

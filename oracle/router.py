@@ -11,13 +11,21 @@ import numpy as np
 from .bf16 import widen
 
 
+def segment_bounds(H: int, parts: int = 4):
+    """h ranges of the partial chains: [floor(q*H/parts), floor((q+1)*H/parts))."""
+    return [(q * H // parts, (q + 1) * H // parts) for q in range(parts)]
+
+
 def router_logits(x_bits: np.ndarray, w_bits: np.ndarray, bias: np.ndarray | None = None) -> np.ndarray:
-    """l[t, e] = sum_h x[t, h] * w[e, h] as an fp32 fused-multiply-add chain over
-    h = 0, 1, ..., H-1 starting from +0, then + bias[e] in one fp32 addition.
+    """l[t, e] = sum_h x[t, h] * w[e, h] in fp32, in this order: four partial
+    sums over the contiguous quarters of h (see segment_bounds), each an fp32
+    fused-multiply-add chain in increasing h starting from +0; then
+    (q0 + q1) + (q2 + q3) in fp32; then + bias[e] in one fp32 addition.
 
     Reading: the routing decision is integer output taken in fp32, so the order
-    of the sum is part of its definition; the plainest order is the sequential
-    one, acc <- fma(x_h, w_h, acc).
+    of the sum is part of its definition; the pages give none. Four contiguous
+    chains combined pairwise are a plain blocked sum whose longest dependency
+    chain is a quarter of the sequential one.
 
     Emulation of fp32 fma in fp64: the product of two bf16 numbers (8-bit
     significands) is exact in fp64, and so is its sum with an fp32 accumulator
@@ -30,12 +38,16 @@ def router_logits(x_bits: np.ndarray, w_bits: np.ndarray, bias: np.ndarray | Non
     w = widen(w_bits)
     T, H = x.shape
     E = w.shape[0]
-    acc = np.zeros((T, E), dtype=np.float32)
-    for h in range(H):
-        acc = (acc.astype(np.float64) + np.outer(x[:, h], w[:, h])).astype(np.float32)
+    part = []
+    for h0, h1 in segment_bounds(H):
+        acc = np.zeros((T, E), dtype=np.float32)
+        for h in range(h0, h1):
+            acc = (acc.astype(np.float64) + np.outer(x[:, h], w[:, h])).astype(np.float32)
+        part.append(acc)
+    logits = (part[0] + part[1]) + (part[2] + part[3])  # fp32 + fp32 -> fp32
     if bias is not None:
-        acc = acc + np.asarray(bias, dtype=np.float32)[None, :]  # fp32 + fp32 -> fp32
-    return acc.astype(np.float32)
+        logits = logits + np.asarray(bias, dtype=np.float32)[None, :]
+    return logits.astype(np.float32)
 
 
 def softmax_gates(logits: np.ndarray) -> np.ndarray:

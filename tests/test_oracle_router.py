@@ -55,12 +55,16 @@ def test_router_logits_match_libm_fmaf_chain():
     got = oracle.router_logits(xb, wb, bias)
     xf = si.bf16_bits_to_f32(xb)
     wf = si.bf16_bits_to_f32(wb)
+    f32 = np.float32
     for t in range(T):
         for e in range(E):
-            acc = ctypes.c_float(0.0).value
-            for h in range(H):
-                acc = libm.fmaf(float(xf[t, h]), float(wf[e, h]), acc)
-            want = np.float32(np.float32(acc) + bias[e])
+            q = []
+            for h0, h1 in [(0, 15), (15, 30), (30, 45), (45, 61)]:  # quarters of 61, floor(q*61/4)
+                acc = 0.0
+                for h in range(h0, h1):
+                    acc = libm.fmaf(float(xf[t, h]), float(wf[e, h]), acc)
+                q.append(f32(acc))
+            want = f32(f32(f32(q[0] + q[1]) + f32(q[2] + q[3])) + bias[e])
             assert np.float32(got[t, e]).view(np.uint32) == want.view(np.uint32), (t, e)
 
 
@@ -71,8 +75,9 @@ def test_router_logits_fma_at_a_double_rounding_boundary():
     own it becomes 1 unit, and acc + 1 unit is a tie that rounds back to 2^-125;
     fma rounds the exact sum up to 2^-125 + 2^-148."""
     f = np.array
-    x = si.f32_to_bf16_bits(f([[2.0 ** -62, 1.5 * 2.0 ** -75]], dtype=np.float32))
-    w = si.f32_to_bf16_bits(f([[2.0 ** -63, (255 / 256) * 2.0 ** -74]], dtype=np.float32))
+    # H = 8: both terms sit in the first quarter (h = 0, 1); the rest are zero
+    x = si.f32_to_bf16_bits(f([[2.0 ** -62, 1.5 * 2.0 ** -75] + [0.0] * 6], dtype=np.float32))
+    w = si.f32_to_bf16_bits(f([[2.0 ** -63, (255 / 256) * 2.0 ** -74] + [0.0] * 6], dtype=np.float32))
     got = oracle.router_logits(x, w)[0, 0]
     assert got == np.float32(2.0 ** -125 + 2.0 ** -148)
     libm = ctypes.CDLL(ctypes.util.find_library("m"))
@@ -80,6 +85,20 @@ def test_router_logits_fma_at_a_double_rounding_boundary():
     libm.fmaf.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_float]
     acc = libm.fmaf(2.0 ** -62, 2.0 ** -63, 0.0)
     assert np.float32(libm.fmaf(1.5 * 2.0 ** -75, (255 / 256) * 2.0 ** -74, acc)) == got
+
+
+def test_router_summation_order_is_the_quarter_tree():
+    """A case that separates the quarter tree from one sequential chain (H = 8,
+    quarters {0,1} {2,3} {4,5} {6,7}): with x = [2^-30, 0, 0, 0, 1, 0, -1, 0]
+    and w = 1, the tree gives (2^-30 + 0) + (1 + -1) = 2^-30, while a single
+    chain absorbs 2^-30 into 1 and ends at 0."""
+    H = 8
+    tiny = 2.0 ** -30
+    x = si.f32_to_bf16_bits(np.array([[tiny, 0, 0, 0, 1.0, 0, -1.0, 0]], dtype=np.float32))
+    w = si.f32_to_bf16_bits(np.ones((1, H), dtype=np.float32))
+    assert oracle.router_logits(x, w)[0, 0] == np.float32(tiny)
+    assert oracle.segment_bounds(1280) == [(0, 320), (320, 640), (640, 960), (960, 1280)]
+    assert oracle.segment_bounds(61) == [(0, 15), (15, 30), (30, 45), (45, 61)]
 
 
 def test_topk_matches_bruteforce_with_ties():
