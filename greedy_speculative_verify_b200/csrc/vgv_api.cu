@@ -20,6 +20,7 @@ namespace {
 
 constexpr int kH = 1280, kI = 896, kE = 64, kS = 2, kTopK = 6;
 constexpr int kMaxDevices = 64;
+constexpr int kEntryMaxGrid = 256;  // CTAs of the layer-entry kernel at most
 
 struct DevState {
   bool init = false;
@@ -88,7 +89,7 @@ vg_status device_state(DevState** out) {
                              vg::FgCfg<64>::kSmemBytes) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::moe_layer_entry<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::layer_entry_smem(kH, vg::kSortSmallMax)) != cudaSuccess)
+                             vg::layer_entry_smem(kH)) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
@@ -130,7 +131,7 @@ bool dims_supported(const vg_moe_dims* d) {
 }
 
 struct MoeWs {
-  size_t idx, w, logits, offsets, perm, inv, xperm, act, o, ccnt, cbase, sched, gbar, total;
+  size_t idx, w, logits, offsets, perm, inv, xperm, act, o, ccnt, cbase, ecnt, sched, gbar, total;
   int sched_len;
 };
 
@@ -163,6 +164,7 @@ MoeWs moe_layout(int T) {
   L.o = take((size_t)(kTopK + kS) * T * kH * 2);
   L.ccnt = take(nch * kE * 4);
   L.cbase = take(nch * kE * 4);
+  L.ecnt = take((size_t)kEntryMaxGrid * kE * 4);
   L.sched_len = 1 + max_tiles(T);
   L.sched = take((size_t)L.sched_len * 4);
   L.gbar = take(8);
@@ -177,7 +179,7 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 // Device buffers of one layer inside the workspace (or the caller's taps).
 struct LayerBufs {
-  int32_t *idx, *offsets, *perm, *inv, *sched, *ccnt, *cbase;
+  int32_t *idx, *offsets, *perm, *inv, *sched, *ccnt, *cbase, *ecnt;
   float *gw, *logits;
   uint32_t* gbar;
   __nv_bfloat16 *xperm, *act, *o;
@@ -202,11 +204,19 @@ LayerBufs carve(void* workspace, int T, const vg_moe_taps* taps) {
   b.sched_len = L.sched_len;
   b.ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
   b.cbase = reinterpret_cast<int32_t*>(ws + L.cbase);
+  b.ecnt = reinterpret_cast<int32_t*>(ws + L.ecnt);
   b.gbar = reinterpret_cast<uint32_t*>(ws + L.gbar);
   return b;
 }
 
-bool small_path(int T) { return (int64_t)T * kTopK <= vg::kSortSmallMax; }
+// The layer-entry kernel takes decode sizes: at most kEntryMaxOwn tokens per CTA
+// of its cooperative grid.
+int entry_grid(const DevState* dev, int T) {
+  return std::min(std::min(dev->sms, kEntryMaxGrid), vg::cdiv(T, vg::kEntryTok));
+}
+bool small_path(const DevState* dev, int T) {
+  return (int64_t)T * kTopK <= vg::kSortSmallMax && vg::cdiv(T, entry_grid(dev, T)) <= vg::kEntryMaxOwn;
+}
 
 // The previous layer's combine, when it is folded into this layer's entry.
 struct PrevCombine {
@@ -218,12 +228,17 @@ struct PrevCombine {
 // `prev` when given: decode path only). Large token counts: separate kernels.
 // `nbar` counts the grid barriers passed on b.gbar since it was zeroed (host side:
 // every launch passes the same number, so it is known without reading the device).
+// Bytes of expert weights the layer entry prefetches into L2: the gate|up rows
+// of the first routed experts, which the expert kernel's first wave of units
+// streams (about one unit per SM).
+constexpr size_t kEntryPrefetchBytes = (size_t)96 << 20;
+
 vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv_bfloat16* x_in,
-                       __nv_bfloat16* x_out, const void* router_w, const float* router_bias, const LayerBufs& b,
-                       uint32_t* nbar, cudaStream_t s) {
+                       __nv_bfloat16* x_out, const void* router_w, const float* router_bias, const void* expert_w,
+                       const LayerBufs& b, uint32_t* nbar, cudaStream_t s) {
   using namespace vg;
   const int N = T * kTopK;
-  if (small_path(T)) {
+  if (small_path(dev, T)) {
     EntryArgs a{};
     if (prev) {
       a.prev_o = prev->b->o;
@@ -234,29 +249,33 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
       a.x_out = x_out;
     }
     a.x_in = x_in;
-    a.w = static_cast<const __nv_bfloat16*>(router_w);
     a.bias = router_bias;
     a.T = T;
     a.H = kH;
     a.k = kTopK;
     a.S = kS;
-    a.logits = b.logits;
     a.idx = b.idx;
     a.gate = b.gw;
     a.offsets = b.offsets;
     a.perm = b.perm;
     a.inv = b.inv;
     a.x_perm = b.xperm;
+    a.counts = b.ecnt;
     a.sched = b.sched;
     a.sched_len = b.sched_len;
     a.gbar = b.gbar;
     a.gbar_base = *nbar;
-    const int grid = min(dev->sms, cdiv(T, kEntryTok));
-    if (grid > 1) *nbar += prev ? 2 : 1;
+    const size_t gu_bytes = (size_t)2 * kI * kH * 2;
+    a.prefetch_base = static_cast<const uint8_t*>(expert_w);
+    a.n_prefetch = (int)min((size_t)kE, kEntryPrefetchBytes / gu_bytes);
+    a.prefetch_bytes = (uint32_t)gu_bytes;
+    a.prefetch_stride = (uint64_t)3 * kI * kH * 2;
+    const int grid = entry_grid(dev, T);
+    if (grid > 1) *nbar += 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kEntryThreads);
-    cfg.dynamicSmemBytes = layer_entry_smem(kH, N);
+    cfg.dynamicSmemBytes = layer_entry_smem(kH);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -357,7 +376,7 @@ vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, 
   if (cudaMemsetAsync(b.gbar, 0, 8, s) != cudaSuccess) return cuda_fail();
   uint32_t nbar = 0;
   vg_status st = launch_entry(dev, T, nullptr, static_cast<const __nv_bfloat16*>(x), nullptr, router_w, router_bias,
-                              b, &nbar, s);
+                              expert_w, b, &nbar, s);
   if (st == VG_OK) st = launch_experts(dev, T, x, expert_w, shared_w, b, s);
   if (st == VG_OK) st = launch_combine(T, x, b, add_residual, out, s);
   return st;
@@ -465,7 +484,7 @@ vg_status vg_moe_ffn_stack(const vg_moe_dims* dims, int32_t n_layers, int32_t T,
       xl = xout;
     }
     st = launch_entry(dev, T, l > 0 ? &prev : nullptr, xin, xout, router_w[l], router_bias ? router_bias[l] : nullptr,
-                      b, &nbar, s);
+                      expert_w[l], b, &nbar, s);
     if (st == VG_OK) st = launch_experts(dev, T, xl, expert_w[l], shared_w[l], b, s);
     if (st != VG_OK) return st;
     xin = xl;
