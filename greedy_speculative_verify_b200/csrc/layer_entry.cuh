@@ -16,11 +16,14 @@
 //
 // The router matrix sits in shared memory as H/64 TMA tiles with the 128-byte
 // swizzle, requested at entry so its latency hides behind the combine. Each
-// logit is four quarter fma chains (one thread each: a warp runs one quarter of
-// one token for 32 experts, lane-consecutive experts reading distinct swizzle
-// slots) combined as (q0 + q1) + (q2 + q3). The arithmetic of every phase is
-// the one of the separate kernels (router.cuh, sort.cuh, combine.cuh). The
-// kernel also prefetches into L2 the first weights the expert kernel will
+// logit is four quarter fma chains combined as (q0 + q1) + (q2 + q3), the
+// order of the router's definition (router.cuh). Thread (group, quarter,
+// expert) runs the chains of up to two tokens at once, so each weight pair is
+// unpacked once for both; lane-consecutive experts read distinct swizzle slots.
+// Top-k is a rank count: the logit of expert e of a token is at rank
+// #{e' : l[e'] > l[e] or (l[e'] == l[e] and e' < e)}, which selects by
+// (logit descending, expert ascending) as the separate router kernel does.
+// The kernel also prefetches into L2 the first weights the expert kernel will
 // stream, while HBM is otherwise idle.
 #pragma once
 #include "combine.cuh"
@@ -40,7 +43,7 @@ struct EntryArgs {
   const __nv_bfloat16* x_in;  // layer input (no combine phase)
   __nv_bfloat16* x_out;       // layer input written by the combine phase
   const float* bias;          // [64] or nullptr
-  int32_t T, H, k, S;
+  int32_t T, k, S;
   int32_t* idx;               // [T, k]
   float* gate;                // [T, k]
   int32_t* offsets;           // [65]
@@ -59,28 +62,65 @@ struct EntryArgs {
   uint64_t prefetch_stride;
 };
 
-constexpr int kEntryTok = 2;                             // tokens routed at a time
-constexpr int kEntryThreads = kEntryTok * kRouterE * 4;  // one thread per quarter chain: 512
-constexpr int kEntryMaxOwn = 16;                         // tokens a CTA may own (T <= 16 * grid)
+constexpr int kEntryH = 1280;                          // hidden size of the kernel
+constexpr int kEntryThreads = 512;                     // 2 groups x 4 quarters x 64 experts
+constexpr int kEntryGroupTok = 2;                      // tokens per group and pass
+constexpr int kEntryPassTok = 2 * kEntryGroupTok;      // tokens per pass
+constexpr int kEntryMaxOwn = 12;                       // tokens a CTA may own (T <= 12 * grid)
+constexpr int kEntrySlices = kEntryThreads / kRouterE; // CTA slices in the offsets phase
 
-// Shared memory: router tiles, owned token rows (bf16), the current pair of
-// rows in fp32, plus 1 KB alignment slack.
-__host__ __device__ constexpr int layer_entry_smem(int H) {
-  return 1024 + kRouterE * H * 2 + kEntryMaxOwn * H * 2 + kEntryTok * H * 4;
+// Shared memory: router tiles, owned token rows (bf16), the pass's rows in
+// fp32, plus 1 KB alignment slack.
+__host__ __device__ constexpr int layer_entry_smem() {
+  return 1024 + kRouterE * kEntryH * 2 + kEntryMaxOwn * kEntryH * 2 + kEntryPassTok * kEntryH * 4;
+}
+
+// NT quarter chains (one per token) over the thread's quarter of h; each
+// weight pair is unpacked once for all NT tokens. `wq` is the thread's row in
+// the swizzled tile of its quarter's first 64 columns, `xq` the quarter's
+// first fp32 input of token 0 (token j at + j * kEntryH).
+template <int NT>
+__device__ __forceinline__ void quarter_chains(const uint8_t* wq, int sw, const float* xq, float* acc) {
+  constexpr int kTiles = kEntryH / 4 / 64;  // a quarter spans 5 tiles of 64 columns
+#pragma unroll
+  for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
+#pragma unroll 1
+  for (int m = 0; m < kTiles; ++m) {
+#pragma unroll
+    for (int q8 = 0; q8 < 8; ++q8) {  // 16-byte slot q8 of the row: columns 8 q8 .. 8 q8 + 7
+      const uint4 wv = *reinterpret_cast<const uint4*>(wq + m * 8192 + ((q8 ^ sw) << 4));
+      const float w[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
+                          bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const float4* xv = reinterpret_cast<const float4*>(xq + j * kEntryH + m * 64 + q8 * 8);
+        const float4 x0 = xv[0], x1 = xv[1];
+        acc[j] = __fmaf_rn(x0.x, w[0], acc[j]);
+        acc[j] = __fmaf_rn(x0.y, w[1], acc[j]);
+        acc[j] = __fmaf_rn(x0.z, w[2], acc[j]);
+        acc[j] = __fmaf_rn(x0.w, w[3], acc[j]);
+        acc[j] = __fmaf_rn(x1.x, w[4], acc[j]);
+        acc[j] = __fmaf_rn(x1.y, w[5], acc[j]);
+        acc[j] = __fmaf_rn(x1.z, w[6], acc[j]);
+        acc[j] = __fmaf_rn(x1.w, w[7], acc[j]);
+      }
+    }
+  }
 }
 
 template <int K>
 __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid_constant__ CUtensorMap mR,
                                                                     const EntryArgs a) {
+  constexpr int H = kEntryH, HQ = H / 4;
   extern __shared__ uint8_t esm_raw[];
   uint8_t* esm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 1023) & ~uintptr_t(1023));
-  const int H = a.H, HQ = H / 4;
   uint8_t* ws = esm;                                                              // [H/64][64 rows][128 B]
   __nv_bfloat16* xo = reinterpret_cast<__nv_bfloat16*>(esm + kRouterE * H * 2);   // [own][H]
-  float* xf = reinterpret_cast<float*>(xo + kEntryMaxOwn * H);                    // [kEntryTok][H]
+  float* xf = reinterpret_cast<float*>(xo + kEntryMaxOwn * H);                    // [kEntryPassTok][H]
   __shared__ __align__(8) uint64_t bars[2];                                       // weights, token rows
-  __shared__ float part[4][kEntryTok][kRouterE];                                  // [quarter][token][expert]
-  __shared__ float logit[kEntryTok][kRouterE];
+  __shared__ __align__(16) float part[4][kEntryPassTok][kRouterE];                // [quarter][token][expert]
+  __shared__ float logit[kEntryPassTok][kRouterE];
+  __shared__ float mx_s[kEntryPassTok], sum_s[kEntryPassTok][2];
   __shared__ int32_t idx_s[kEntryMaxOwn * K];
   __shared__ int cnt_s[kRouterE], tot_s[kRouterE], pre_s[kRouterE], off_s[kRouterE];
 
@@ -96,7 +136,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
     fence_mbar_init();
     if (n_own > 0) {  // the router matrix is streamed in while the combine runs
       mbar_arrive_expect_tx(&bars[0], kRouterE * H * 2);
-      const int nkc = H / 64;
+      constexpr int nkc = H / 64;
       for (int i = 0; i < nkc; ++i) {  // CTAs start at different tiles: spread over L2 slices
         const int kc = (i + c) % nkc;
         tma_load_2d(ws + kc * 8192, &mR, &bars[0], kc * 64, 0);
@@ -118,7 +158,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
 
   // ---- A1: this CTA's input rows
   if (a.prev_o != nullptr) {
-    const int per_row = H / 8;
+    constexpr int per_row = H / 8;
     for (int i = tid; i < n_own * per_row; i += blockDim.x) {
       const int tl = i / per_row, cc = i - tl * per_row, t = t_begin + tl;
       const uint4 v = combine8(a.prev_x, a.prev_o, a.prev_inv, a.prev_gate, a.T, H, a.k, a.S, a.prev_add_residual, t, cc);
@@ -141,47 +181,62 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   }
   ok = __syncthreads_and(ok);  // one decision for the whole CTA
 
-  // ---- A2: logits and top-k, kEntryTok tokens at a time
-  const int qq = warp / (2 * kEntryTok), tl = (warp >> 1) % kEntryTok, e = ((warp & 1) << 5) | lane;
-  for (int g0 = 0; ok && g0 < n_own; g0 += kEntryTok) {
-    for (int i = tid; i < kEntryTok * H / 2; i += blockDim.x) {  // the pair's rows to fp32
-      const int r = (2 * i) / H;
-      const uint32_t v = g0 + r < n_own ? reinterpret_cast<const uint32_t*>(xo + (size_t)g0 * H)[i] : 0u;
+  // ---- A2: logits, top-k and gates, kEntryPassTok tokens at a time
+  const int grp = tid >> 8, qq = (tid >> 6) & 3, e = tid & 63;
+  for (int g0 = 0; ok && g0 < n_own; g0 += kEntryPassTok) {
+    const int n_pass = min(kEntryPassTok, n_own - g0);
+    for (int i = tid; i < n_pass * H / 2; i += blockDim.x) {  // the pass's rows to fp32
+      const uint32_t v = reinterpret_cast<const uint32_t*>(xo + (size_t)g0 * H)[i];
       reinterpret_cast<float2*>(xf)[i] = make_float2(bf16_lo(v), bf16_hi(v));
     }
     __syncthreads();
-    const float4* xr = reinterpret_cast<const float4*>(xf + tl * H + qq * HQ);
-    const uint8_t* wrow = ws + e * 128;
-    float acc = 0.0f;
+    const int tok0 = grp * kEntryGroupTok, n_grp = min(kEntryGroupTok, n_pass - tok0);  // warp-uniform
+    if (n_grp > 0) {
+      const uint8_t* wq = ws + qq * (HQ / 64) * 8192 + e * 128;
+      const float* xq = xf + tok0 * H + qq * HQ;
+      float acc[kEntryGroupTok];
+      if (n_grp == 2) {
+        quarter_chains<2>(wq, e & 7, xq, acc);
+        part[qq][tok0 + 1][e] = acc[1];
+      } else {
+        quarter_chains<1>(wq, e & 7, xq, acc);
+      }
+      part[qq][tok0][e] = acc[0];
+    }
+    __syncthreads();
+    const int tk = tid >> 6;  // (token, expert) threads for the rest of the pass
+    float l = 0.0f;
+    int rank = kRouterE;
+    if (tk < n_pass) {
+      l = (part[0][tk][e] + part[1][tk][e]) + (part[2][tk][e] + part[3][tk][e]);
+      if (a.bias != nullptr) l = __fadd_rn(l, a.bias[e]);
+      logit[tk][e] = l;
+    }
+    __syncthreads();
+    if (tk < n_pass) {
+      rank = 0;
 #pragma unroll 8
-    for (int p = 0; p < HQ / 8; ++p) {
-      const int kk = qq * HQ + p * 8;  // 8 consecutive k in one 16-byte slot
-      const int kc = kk >> 6, j = (kk >> 3) & 7;
-      const uint4 wv = *reinterpret_cast<const uint4*>(wrow + kc * 8192 + ((j ^ (e & 7)) << 4));
-      const float4 x0 = xr[2 * p], x1 = xr[2 * p + 1];
-      acc = __fmaf_rn(x0.x, bf16_lo(wv.x), acc);
-      acc = __fmaf_rn(x0.y, bf16_hi(wv.x), acc);
-      acc = __fmaf_rn(x0.z, bf16_lo(wv.y), acc);
-      acc = __fmaf_rn(x0.w, bf16_hi(wv.y), acc);
-      acc = __fmaf_rn(x1.x, bf16_lo(wv.z), acc);
-      acc = __fmaf_rn(x1.y, bf16_hi(wv.z), acc);
-      acc = __fmaf_rn(x1.z, bf16_lo(wv.w), acc);
-      acc = __fmaf_rn(x1.w, bf16_hi(wv.w), acc);
-    }
-    part[qq][tl][e] = acc;
-    __syncthreads();
-    if (tid < kEntryTok * kRouterE) {
-      const int t2 = tid >> 6, e2 = tid & 63;
-      float l = (part[0][t2][e2] + part[1][t2][e2]) + (part[2][t2][e2] + part[3][t2][e2]);
-      if (a.bias != nullptr) l = __fadd_rn(l, a.bias[e2]);
-      logit[t2][e2] = l;
+      for (int j = 0; j < kRouterE; ++j) {
+        const float o = logit[tk][j];
+        rank += (o > l || (o == l && j < e)) ? 1 : 0;
+      }
+      if (rank == 0) mx_s[tk] = l;
     }
     __syncthreads();
-    if (warp < kEntryTok && g0 + warp < n_own) {
-      const int own = g0 + warp, t = t_begin + own;
-      topk_softmax_warp<K>(logit[warp], lane, idx_s + own * K, a.gate + (size_t)t * K);
-      __syncwarp();
-      if (lane < K) a.idx[(size_t)t * K + lane] = idx_s[own * K + lane];
+    float ex = 0.0f;
+    if (tk < n_pass) {
+      ex = expf(l - mx_s[tk]);
+      float s = ex;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) sum_s[tk][(tid >> 5) & 1] = s;
+    }
+    __syncthreads();
+    if (tk < n_pass && rank < K) {
+      const int own = g0 + tk, t = t_begin + own;
+      idx_s[own * K + rank] = e;
+      a.idx[(size_t)t * K + rank] = e;
+      a.gate[(size_t)t * K + rank] = ex / (sum_s[tk][0] + sum_s[tk][1]);
     }
     __syncthreads();
   }
@@ -200,21 +255,28 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   if (!ok) return;
 
   // ---- B: offsets, positions of this CTA's assignments, rows to their positions
-  for (int ee = warp; ee < kRouterE; ee += blockDim.x / 32) {
+  {
+    int* red = reinterpret_cast<int*>(&part[0][0][0]);  // [2][kEntrySlices][64]
+    const int s = tid >> 6;
     int tot = 0, pre = 0;
-    for (int cc = lane; cc < G; cc += 32) {
-      const int v = __ldcg(a.counts + (size_t)cc * kRouterE + ee);
+#pragma unroll 4
+    for (int cc = s; cc < G; cc += kEntrySlices) {
+      const int v = __ldcg(a.counts + (size_t)cc * kRouterE + e);
       tot += v;
       pre += cc < c ? v : 0;
     }
+    red[s * kRouterE + e] = tot;
+    red[(kEntrySlices + s) * kRouterE + e] = pre;
+    __syncthreads();
+    if (tid < kRouterE) {
+      int t2 = 0, p2 = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      tot += __shfl_xor_sync(0xffffffffu, tot, o);
-      pre += __shfl_xor_sync(0xffffffffu, pre, o);
-    }
-    if (lane == 0) {
-      tot_s[ee] = tot;
-      pre_s[ee] = pre;
+      for (int j = 0; j < kEntrySlices; ++j) {
+        t2 += red[j * kRouterE + tid];
+        p2 += red[(kEntrySlices + j) * kRouterE + tid];
+      }
+      tot_s[tid] = t2;
+      pre_s[tid] = p2;
     }
   }
   __syncthreads();

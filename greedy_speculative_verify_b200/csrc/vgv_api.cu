@@ -89,7 +89,7 @@ vg_status device_state(DevState** out) {
                              vg::FgCfg<64>::kSmemBytes) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::moe_layer_entry<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::layer_entry_smem(kH)) != cudaSuccess)
+                             vg::layer_entry_smem()) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
@@ -212,7 +212,7 @@ LayerBufs carve(void* workspace, int T, const vg_moe_taps* taps) {
 // The layer-entry kernel takes decode sizes: at most kEntryMaxOwn tokens per CTA
 // of its cooperative grid.
 int entry_grid(const DevState* dev, int T) {
-  return std::min(std::min(dev->sms, kEntryMaxGrid), vg::cdiv(T, vg::kEntryTok));
+  return std::min(std::min(dev->sms, kEntryMaxGrid), T);
 }
 bool small_path(const DevState* dev, int T) {
   return (int64_t)T * kTopK <= vg::kSortSmallMax && vg::cdiv(T, entry_grid(dev, T)) <= vg::kEntryMaxOwn;
@@ -251,7 +251,6 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     a.x_in = x_in;
     a.bias = router_bias;
     a.T = T;
-    a.H = kH;
     a.k = kTopK;
     a.S = kS;
     a.idx = b.idx;
@@ -275,7 +274,7 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kEntryThreads);
-    cfg.dynamicSmemBytes = layer_entry_smem(kH);
+    cfg.dynamicSmemBytes = layer_entry_smem();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
