@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(256) moe_combine(const __nv_bfloat16* __restri
                                                    const int32_t* __restrict__ inv, const float* __restrict__ g,
                                                    int T, int H, int k, int S, int add_residual,
                                                    __nv_bfloat16* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int per_row = H / 8;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T * per_row) return;

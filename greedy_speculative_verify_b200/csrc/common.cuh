@@ -239,6 +239,17 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* ctr, uint32_t target, uin
   return ok_s != 0;
 }
 
+// ----------------------------------------------------------------- dependent launch
+// Kernels of the decode path are launched with programmatic stream
+// serialization: one may start while its predecessor in the stream is still
+// running. griddep_wait() returns once the predecessor grid has completed and
+// its memory is visible; every thread calls it before touching global data the
+// predecessor writes or reads (reading immutable weights before it is fine).
+// griddep_launch_dependents() lets the successor be scheduled on SMs as they
+// free up, so its launch and prologue overlap this kernel's tail.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------- misc
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_exp = args.E + args.S;
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  griddep_wait();  // barriers, tensor maps and TMEM are set up; the grouping is read from here on
   if (warp == 2) {
     const int kT = args.offsets[args.E];
     for (int e = lane; e < n_exp; e += 32) {

@@ -24,7 +24,8 @@
 // #{e' : l[e'] > l[e] or (l[e'] == l[e] and e' < e)}, which selects by
 // (logit descending, expert ascending) as the separate router kernel does.
 // The kernel also prefetches into L2 the first weights the expert kernel will
-// stream, while HBM is otherwise idle.
+// stream, while HBM is otherwise idle. Both the router tiles and the prefetch
+// are requested before waiting for the previous kernel (dependent launch).
 #pragma once
 #include "combine.cuh"
 #include "common.cuh"
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   const int P = cdiv(a.T, G);
   const int t_begin = min(a.T, c * P), t_end = min(a.T, t_begin + P), n_own = t_end - t_begin;
 
+  griddep_launch_dependents();
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -154,6 +156,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   }
   if (tid < kRouterE) cnt_s[tid] = 0;
   __syncthreads();
+  griddep_wait();  // the router tiles and the L2 prefetch are under way; now the previous kernel's data
   bool ok = true;
 
   // ---- A1: this CTA's input rows

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kLmStages; ++i) {
       mbar_init(&full[i], 1);
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the hidden states come from the previous kernel
   const uint32_t tmem_base = *tmem_slot;
   const int total = n_groups * n_mblk;  // unit = (vocabulary group, row block), row block fastest
   const uint64_t limit = g_wait_timeout_ns;
@@ -234,6 +236,8 @@ __global__ void __launch_bounds__(1024) argmax_accept(const uint64_t* __restrict
                                                       int32_t* __restrict__ argmax, int32_t* __restrict__ accepted,
                                                       int32_t* __restrict__ out_tokens) {
   __shared__ int32_t arg_s[256];
+  griddep_launch_dependents();
+  griddep_wait();
   const int spb = max(1, 32 / (K + 1));
   const int seq0 = blockIdx.x * spb;
   const int nseq = min(spb, B - seq0);

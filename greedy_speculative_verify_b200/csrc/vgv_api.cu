@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "vgv.h"
@@ -233,6 +234,27 @@ struct PrevCombine {
 // streams (about one unit per SM).
 constexpr size_t kEntryPrefetchBytes = (size_t)96 << 20;
 
+// Launch of a decode-path kernel with programmatic stream serialization (the
+// kernel waits for its predecessor itself, see griddep_wait), optionally
+// cooperative.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, bool coop,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = coop ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv_bfloat16* x_in,
                        __nv_bfloat16* x_out, const void* router_w, const float* router_bias, const void* expert_w,
                        const LayerBufs& b, uint32_t* nbar, cudaStream_t s) {
@@ -271,22 +293,13 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     a.prefetch_stride = (uint64_t)3 * kI * kH * 2;
     const int grid = entry_grid(dev, T);
     if (grid > 1) *nbar += 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kEntryThreads);
-    cfg.dynamicSmemBytes = layer_entry_smem();
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     CUtensorMap mR;
     const uint64_t dR[2] = {kH, kE}, sR[1] = {kH * 2};
     const uint32_t bR[2] = {64, kE};
     if (make_map(&mR, router_w, 2, dR, sR, bR)) return VG_ERR_CUDA;
     ProfScope ps(VG_KERNEL_ROUTER, s);
-    if (cudaLaunchKernelEx(&cfg, moe_layer_entry<kTopK>, mR, a) != cudaSuccess) return cuda_fail();
+    if (launch_dep(moe_layer_entry<kTopK>, grid, kEntryThreads, layer_entry_smem(), s, true, mR, a) != cudaSuccess)
+      return cuda_fail();
     return VG_OK;
   }
   const __nv_bfloat16* xcur = x_in;
@@ -352,19 +365,23 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   a.out = b.o;
   const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
   ProfScope ps(VG_KERNEL_EXPERTS, s);
-  if (expert_tile(T) == 64)
-    moe_expert_gemms<64><<<grid, 192, FgCfg<64>::kSmemBytes, s>>>(mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct, a);
-  else
-    moe_expert_gemms<128><<<grid, 192, FgCfg<128>::kSmemBytes, s>>>(mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct, a);
-  return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+  const cudaError_t e =
+      expert_tile(T) == 64
+          ? launch_dep(moe_expert_gemms<64>, grid, 192, FgCfg<64>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS, mXr,
+                       mXs, mAct, a)
+          : launch_dep(moe_expert_gemms<128>, grid, 192, FgCfg<128>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS,
+                       mXr, mXs, mAct, a);
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
 }
 
 vg_status launch_combine(int T, const void* x, const LayerBufs& b, int add_residual, void* out, cudaStream_t s) {
   using namespace vg;
   ProfScope ps(VG_KERNEL_COMBINE, s);
-  moe_combine<<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), b.o, b.inv, b.gw, T, kH,
-                                                     kTopK, kS, add_residual, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+  const cudaError_t e = launch_dep(moe_combine, cdiv(T * (kH / 8), 256), 256, 0, s, false,
+                                   static_cast<const __nv_bfloat16*>(x), (const __nv_bfloat16*)b.o,
+                                   (const int32_t*)b.inv, (const float*)b.gw, T, kH, kTopK, kS, add_residual,
+                                   static_cast<__nv_bfloat16*>(out));
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
 }
 
 // One layer: entry, expert GEMMs, combine into out.
@@ -530,16 +547,17 @@ vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V, const voi
   const int grid = min(dev->sms, n_mblk * n_groups);
   {
   ProfScope ps(VG_KERNEL_LM_HEAD, s);
-  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, kLmGroupTiles, n_groups,
-                                                a_box_rows, box_rows(V, kLmN), part);
+  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, false, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
+                 kLmGroupTiles, n_groups, a_box_rows, box_rows(V, kLmN), part) != cudaSuccess)
+    return VG_ERR_CUDA;
   }
-  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   const int spb = max(1, 32 / (K + 1));
   {
     ProfScope ps(VG_KERNEL_ACCEPT, s);
-    argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_groups, R, B, K, drafts, argmax, accepted, out_tokens);
+    if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, false, (const uint64_t*)part, n_groups, R, B, K, drafts,
+                   argmax, accepted, out_tokens) != cudaSuccess)
+      return VG_ERR_CUDA;
   }
-  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   return VG_OK;
 }
 
@@ -659,11 +677,12 @@ extern "C" vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, i
     if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
   }
   const int grid = min(dev->sms, n_mblk * n_groups);
-  lmhead_argmax<<<grid, 192, kLmSmemBytes, s>>>(mH, mLM, R, V, H / kBK, n_mblk, n_vblk, kLmGroupTiles, n_groups,
-                                                a_box_rows, box_rows(V, kLmN), part);
-  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, false, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
+                 kLmGroupTiles, n_groups, a_box_rows, box_rows(V, kLmN), part) != cudaSuccess)
+    return VG_ERR_CUDA;
   const int spb = max(1, 32 / (K + 1));
-  argmax_accept<<<cdiv(B, spb), 1024, 0, s>>>(part, n_groups, R, B, K, drafts, argmax, accepted, out_tokens);
-  if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
+  if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, false, (const uint64_t*)part, n_groups, R, B, K, drafts,
+                 argmax, accepted, out_tokens) != cudaSuccess)
+    return VG_ERR_CUDA;
   return VG_OK;
 }
