@@ -2,31 +2,36 @@
 // SwiGLU epilogue and down, in one persistent launch.
 //
 // Orientation ("swap AB"): the weight rows are the M = 128 operand (A) and the
-// tokens routed to an expert are the N operand (B), so one tile streams a
-// 128-row slab of one expert's weights once for all of that expert's tokens
-// (up to 128 per tile). At decode sizes (about 12 tokens per expert) this is a
-// weight stream bound by HBM; at prefill sizes (thousands of tokens per expert)
-// the same kernel runs full 128 x 128 tiles and is bound by the tensor pipe.
+// tokens routed to an expert are the N operand (B), so one tile streams a slab
+// of one expert's weights once for all of that expert's tokens (up to NMAX per
+// tile). At decode sizes (about 12 tokens per expert) this is a weight stream
+// bound by HBM; at prefill sizes (thousands of tokens per expert) the same
+// kernel runs full 128 x 128 tiles and is bound by the tensor pipe.
 //
-//   gate/up unit: D_gate = W_gate[rows] X^T, D_up = W_up[rows] X^T,
-//                 act[token, row] = bf16(silu(D_gate) * D_up)
-//   down unit:    D = W_down[rows] act^T, out[token, row] = bf16(D)
+// Every pipeline stage carries two 128 x 64 weight tiles (32 KB, one TMA
+// instruction) and one 64-wide k-chunk of the tile's token rows, and feeds two
+// accumulators that share the token operand:
+//   gate/up unit (tile, 128-row block r): the gate and up rows of block r
+//       (one box of a 4-d view: k, row, gate|up, expert) into D0 = gate,
+//       D1 = up; act[token, r rows] = bf16(silu(D0) * D1);
+//   down unit (tile, 256-row block r): rows 256 r .. 256 r + 255 of W_down (one
+//       256-row box) into D0 = lower, D1 = upper 128 rows; out[token, rows] = bf16(D).
 //
 // Token tiles: each expert's tokens (its segment of the permutation; all T
 // tokens for the two shared experts, which ride along as experts E and E+1)
-// are cut into tiles of up to 128. Units are (tile, 128-row block): first all
-// gate/up units, then all down units. CTAs are persistent and take units from
-// a global ticket counter, so no SM idles while units remain. A down unit needs
-// the activations of its tile, i.e. all gate/up units of that tile: their
-// epilogues count up a per-tile readiness word (release), and the producer of a
-// down unit first streams the unit's weights into the free pipeline stages and
-// only then waits (acquire, bounded) for the readiness word before loading the
-// activations. Tickets are handed out in order and only to running CTAs, so a
-// waited-for unit is always already running somewhere: no deadlock, no
-// assumption about co-residency.
+// are cut into tiles of up to NMAX. Units are first all gate/up units, then all
+// down units. CTAs are persistent and take units from a global ticket counter,
+// so no SM idles while units remain. A down unit needs the activations of its
+// tile, i.e. all gate/up units of that tile: their epilogues count up a
+// per-tile readiness word (release), and the producer of a down unit first
+// streams the unit's weights into the free pipeline stages and only then waits
+// (acquire, bounded) for the readiness word before loading the activations.
+// Tickets are handed out in order and only to running CTAs, so a waited-for
+// unit is always already running somewhere: no deadlock, no assumption about
+// co-residency.
 //
-// Warp roles (192 threads): warp 0 takes tickets and issues TMA loads into a
-// 4-stage ring; warp 1 owns the tensor memory and one of its threads issues
+// Warp roles (192 threads): warp 0 takes tickets and issues TMA loads into the
+// stage ring; warp 1 owns the tensor memory and one of its threads issues
 // tcgen05.mma; warps 2-5 drain the double-buffered TMEM accumulator (each warp
 // its own 32-lane quarter) and store the epilogue. Every wait is bounded; a
 // timeout records VG_ERR_TIMEOUT, the CTA drains its in-flight copies and MMAs
@@ -36,41 +41,38 @@
 
 namespace vg {
 
-constexpr int kBM = 128;       // weight rows per tile
+constexpr int kBM = 128;       // weight rows per MMA tile
 constexpr int kBK = 64;        // K elements per stage: one 128-byte swizzle row
 constexpr int kNMax = 128;     // tokens per tile, widest configuration
-constexpr int kBoxRows = 16;   // token rows per TMA box of the B operand
+constexpr int kBoxRows = 32;   // token rows per TMA box of the B operand
 constexpr int kMaxExperts = 72;
 
 // Two configurations of the same kernel, by tile width NMAX:
 //  * NMAX = 128, 4 stages: prefill-sized expert segments, 128 x 128 tiles;
 //  * NMAX = 64, 5 stages: decode sizes, where the token slot of a stage is
 //    small and the freed shared memory buys a fifth stage of weights in flight.
-// A stage holds two 16 KB weight tiles and an NMAX x 64 token slot.
 template <int NMAX>
 struct FgCfg {
   static constexpr int kStages = NMAX == 128 ? 4 : 5;
-  static constexpr int kABytes = kBM * kBK * 2;          // 16 KB
+  static constexpr int kABytes = 2 * kBM * kBK * 2;      // two 16 KB weight tiles
   static constexpr int kBBytes = NMAX * kBK * 2;         // token slot
-  static constexpr int kStageBytes = 2 * kABytes + kBBytes;
-  static constexpr int kAccCols = 2 * NMAX;              // one accumulator buffer (gate | up)
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kAccCols = 2 * NMAX;              // one accumulator buffer (D0 | D1)
   static constexpr int kTmemCols = 2 * kAccCols;         // double buffered
   static constexpr int kAuxBytes = 2048;
   static constexpr int kSmemBytes = kStages * kStageBytes + kAuxBytes + 1024;  // + alignment slack
-  static constexpr int kPairBOff = kBBytes / 2;          // second k-chunk's token rows in a paired stage
 };
-constexpr int kFgABytes = kBM * kBK * 2;
+constexpr int kFgTileBytes = kBM * kBK * 2;               // one 128 x 64 weight tile
 constexpr int kFgRing = 4;                                // unit-ticket ring between the roles
 constexpr int kFgEpiWarps = 4;
 
 struct FusedArgs {
   const int32_t* offsets;  // [E+1] routed segment offsets in permutation order
   int32_t T, E, S;
-  int32_t mblk_gu;         // I / 128
-  int32_t mblk_dn;         // H / 128
+  int32_t mblk_gu;         // I / 128 gate/up row blocks
+  int32_t mblk_dn;         // H / 256 down row blocks
   int32_t kc_gu;           // H / 64
   int32_t kc_dn;           // I / 64
-  int32_t a_up_row;        // first up row inside an expert's gate|up rows (= I)
   int32_t box_xr, box_xs, box_act;  // rows per B box of each B map
   int32_t* sched;          // [0]: ticket counter, [1 + t]: readiness of tile t; zero at launch
   __nv_bfloat16* act;      // [(k+S)T, I]: routed rows in permutation order, then shared
@@ -100,23 +102,21 @@ __device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, 
   }
   un.tile = v / nm;
   un.mb = v - un.tile * nm;
-  int e = 0;
-  while (e + 1 < n_exp && s.pref[e + 1] <= un.tile) ++e;
+  // the expert of the tile: the last e with pref[e] <= tile (experts without
+  // tokens have pref[e] == pref[e + 1] and are skipped by taking the last)
+  int lo = 0, hi = n_exp - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.pref[mid] <= un.tile) lo = mid;
+    else hi = mid - 1;
+  }
+  const int e = lo;
   const int nb = un.tile - s.pref[e];
   un.e = e;
   un.nrows = min(nmax, s.n[e] - nb * nmax);
   un.xrow = s.xrow[e] + nb * nmax;
   un.arow = s.arow[e] + nb * nmax;
   return un;
-}
-
-// Tiles of at most NMAX/2 tokens put two consecutive k-chunks of one weight
-// matrix in a stage (both 16 KB weight slots, 256 contiguous bytes per weight
-// row; the token slot holds both chunks' rows): down units stream W_down that
-// way; gate/up units alternate a gate stage and an up stage over the same two
-// k-chunks.
-__device__ __forceinline__ bool fg_paired(const FgUnit& un, const FusedArgs& a, int nmax) {
-  return un.nrows <= nmax / 2 && ((un.down ? a.kc_dn : a.kc_gu) & 1) == 0;
 }
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
@@ -126,33 +126,6 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Stages of a unit and the weight tiles of its stage j: (k offset, row) of the
-// first tile, the second tile (k offset, row) or k = -1 if the stage has one.
-struct FgStage {
-  int k0, row0, k1, row1;
-};
-__device__ __forceinline__ int fg_nstages(const FgUnit& un, const FusedArgs& a, bool pair) {
-  const int kcs = un.down ? a.kc_dn : a.kc_gu;
-  return pair ? (un.down ? kcs / 2 : kcs) : kcs;
-}
-__device__ __forceinline__ FgStage fg_stage(const FgUnit& un, const FusedArgs& a, bool pair, int j) {
-  FgStage g;
-  if (pair) {
-    const int kc = un.down ? 2 * j : 2 * (j >> 1);
-    const int row = (!un.down && (j & 1)) ? a.a_up_row + un.mb * kBM : un.mb * kBM;
-    g.k0 = kc * kBK;
-    g.row0 = row;
-    g.k1 = (kc + 1) * kBK;
-    g.row1 = row;
-  } else {
-    g.k0 = j * kBK;
-    g.row0 = un.mb * kBM;
-    g.k1 = un.down ? -1 : j * kBK;
-    g.row1 = a.a_up_row + un.mb * kBM;
-  }
-  return g;
 }
 
 template <int NMAX>
@@ -290,23 +263,13 @@ __global__ void __launch_bounds__(192, 1)
         const int box = un.down ? args.box_act : (shared ? args.box_xs : args.box_xr);
         const int brow0 = un.down ? un.arow : un.xrow;
         const int nbox = cdiv(un.nrows, box);
-        const int kcs = un.down ? args.kc_dn : args.kc_gu;
-        // a down tile of <= 64 tokens carries two consecutive k-chunks per stage
-        const bool pair = fg_paired(un, args, NMAX);
-        // stages of a unit: paired down: kcs/2; paired gate/up: kcs (gate, up, gate, ...); else kcs
-        const int nst = fg_nstages(un, args, pair);
-        const uint32_t bchunk = nbox * box * kBK * 2;
-        const uint32_t bytes = pair ? 2 * kFgABytes + 2 * bchunk : (un.down ? 1 : 2) * kFgABytes + bchunk;
+        const int nst = un.down ? args.kc_dn : args.kc_gu;
+        const int arow = un.down ? un.mb * 2 * kBM : un.mb * kBM;
+        const uint32_t bytes = C::kABytes + nbox * box * kBK * 2;
         bool ok = true;
-        // first k-chunk of stage j
-        auto kc_of = [&](int j) { return pair ? (un.down ? 2 * j : 2 * (j >> 1)) : j; };
-        auto load_b = [&](int st, int j) {
-          uint8_t* bt = tiles + st * C::kStageBytes + 2 * kFgABytes;
-          for (int h = 0; h < (pair ? 2 : 1); ++h) {
-            const int kc = kc_of(j) + h;
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d(bt + h * C::kPairBOff + b * box * kBK * 2, mB, &full[st], kc * kBK, brow0 + b * box);
-          }
+        auto load_b = [&](int st, int kc) {
+          uint8_t* bt = tiles + st * C::kStageBytes + C::kABytes;
+          for (int b = 0; b < nbox; ++b) tma_load_2d(bt + b * box * kBK * 2, mB, &full[st], kc * kBK, brow0 + b * box);
         };
         // weights of the first stages go out before the activations are known to be ready
         const int npre = un.down ? min(C::kStages, nst) : 0;
@@ -320,9 +283,10 @@ __global__ void __launch_bounds__(192, 1)
           }
           uint8_t* st = tiles + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          const FgStage g = fg_stage(un, args, pair, kc);
-          tma_load_3d_hint(st, mA, &full[stage], g.k0, g.row0, ecoord, pol_w);
-          if (g.k1 >= 0) tma_load_3d_hint(st + kFgABytes, mA, &full[stage], g.k1, g.row1, ecoord, pol_w);
+          if (un.down)
+            tma_load_3d_hint(st, mA, &full[stage], kc * kBK, arow, ecoord, pol_w);
+          else
+            tma_load_4d_hint(st, mA, &full[stage], kc * kBK, arow, 0, ecoord, pol_w);
           if (kc >= npre) load_b(stage, kc);
           if (kc + 1 == npre) {
             // every stage of the prefetch holds its weights in flight: now wait for the tile
@@ -377,9 +341,7 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t idesc = idesc_bf16_f32(kBM, cdiv(un.nrows, 16) * 16);
         const uint32_t d0 = tmem_base + ab * C::kAccCols;
         const uint32_t d1 = d0 + NMAX;
-        const int kcs = un.down ? args.kc_dn : args.kc_gu;
-        const bool pair = fg_paired(un, args, NMAX);
-        const int nst = fg_nstages(un, args, pair);
+        const int nst = un.down ? args.kc_dn : args.kc_gu;
         bool ok = true;
         for (int kc = 0; kc < nst; ++kc) {
           if (!mbar_wait(&full[stage], phase, limit)) {
@@ -391,24 +353,13 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
           const uint32_t st = smem_u32(tiles + stage * C::kStageBytes);
           const uint64_t a0 = sw128_kmajor_desc(st);
-          const uint64_t a1 = sw128_kmajor_desc(st + kFgABytes);
-          const uint64_t b = sw128_kmajor_desc(st + 2 * kFgABytes);
-          if (pair) {
-            // down: stage kc accumulates into d0; gate/up: even stages gate (d0), odd up (d1)
-            const uint64_t b1 = sw128_kmajor_desc(st + 2 * kFgABytes + C::kPairBOff);
-            const uint32_t d = (!un.down && (kc & 1)) ? d1 : d0;
-            const uint32_t first = un.down ? (kc == 0) : (kc < 2);
+          const uint64_t a1 = sw128_kmajor_desc(st + kFgTileBytes);
+          const uint64_t b = sw128_kmajor_desc(st + C::kABytes);
 #pragma unroll
-            for (int k16 = 0; k16 < kBK / 16; ++k16) umma_bf16(d, a0 + 2 * k16, b + 2 * k16, idesc, !(first && k16 == 0));
-#pragma unroll
-            for (int k16 = 0; k16 < kBK / 16; ++k16) umma_bf16(d, a1 + 2 * k16, b1 + 2 * k16, idesc, 1);
-          } else {
-#pragma unroll
-            for (int k16 = 0; k16 < kBK / 16; ++k16) {
-              const uint32_t acc = (kc | k16) != 0;
-              umma_bf16(d0, a0 + 2 * k16, b + 2 * k16, idesc, acc);
-              if (!un.down) umma_bf16(d1, a1 + 2 * k16, b + 2 * k16, idesc, acc);
-            }
+          for (int k16 = 0; k16 < kBK / 16; ++k16) {
+            const uint32_t acc = (kc | k16) != 0;
+            umma_bf16(d0, a0 + 2 * k16, b + 2 * k16, idesc, acc);
+            umma_bf16(d1, a1 + 2 * k16, b + 2 * k16, idesc, acc);
           }
           umma_commit(&empty[stage]);
           if (++stage == C::kStages) {
@@ -453,19 +404,34 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + ab * C::kAccCols;
-      const int ld = un.down ? args.mblk_dn * kBM : args.mblk_gu * kBM;
-      __nv_bfloat16* dst = (un.down ? args.out : args.act) + (size_t)un.arow * ld + un.mb * kBM + row;
-      for (int c0 = 0; c0 < un.nrows; c0 += 16) {
-        uint32_t g[16], v[16];
-        tmem_ld16(t0 + c0, g);
-        if (!un.down) tmem_ld16(t0 + NMAX + c0, v);
-        tmem_ld_wait();
+      if (un.down) {
+        const int ld = args.mblk_dn * 2 * kBM;
+        __nv_bfloat16* dst = args.out + (size_t)un.arow * ld + un.mb * 2 * kBM + row;
+        for (int c0 = 0; c0 < un.nrows; c0 += 16) {
+          uint32_t g[16], v[16];
+          tmem_ld16(t0 + c0, g);
+          tmem_ld16(t0 + NMAX + c0, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (c0 + j < un.nrows) {
-            const float r = un.down ? __uint_as_float(g[j]) : silu(__uint_as_float(g[j])) * __uint_as_float(v[j]);
-            dst[(size_t)(c0 + j) * ld] = __float2bfloat16_rn(r);
+          for (int j = 0; j < 16; ++j) {
+            if (c0 + j < un.nrows) {
+              dst[(size_t)(c0 + j) * ld] = __float2bfloat16_rn(__uint_as_float(g[j]));
+              dst[(size_t)(c0 + j) * ld + kBM] = __float2bfloat16_rn(__uint_as_float(v[j]));
+            }
           }
+        }
+      } else {
+        const int ld = args.mblk_gu * kBM;
+        __nv_bfloat16* dst = args.act + (size_t)un.arow * ld + un.mb * kBM + row;
+        for (int c0 = 0; c0 < un.nrows; c0 += 16) {
+          uint32_t g[16], v[16];
+          tmem_ld16(t0 + c0, g);
+          tmem_ld16(t0 + NMAX + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < un.nrows)
+              dst[(size_t)(c0 + j) * ld] = __float2bfloat16_rn(silu(__uint_as_float(g[j])) * __uint_as_float(v[j]));
         }
       }
       tc_fence_before();

@@ -112,7 +112,7 @@ vg_status device_state(DevState** out) {
 // bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes.
 vg_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
                    const uint32_t* box) {
-  uint32_t estr[3] = {1, 1, 1};
+  uint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -334,16 +334,20 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   const __nv_bfloat16* dr = static_cast<const __nv_bfloat16*>(expert_w) + (size_t)2 * kI * kH;
   const __nv_bfloat16* dsh = static_cast<const __nv_bfloat16*>(shared_w) + (size_t)2 * kI * kH;
   CUtensorMap mGuR, mGuS, mDnR, mDnS, mXr, mXs, mAct;
-  const uint64_t dGu[3] = {kH, 2 * kI, kE}, dGuS[3] = {kH, 2 * kI, kS}, sGu[2] = {kH * 2, estride};
+  // gate/up as (k, row, gate|up, expert): one box = the gate and up tiles of a row block
+  const uint64_t dGu[4] = {kH, kI, 2, kE}, dGuS[4] = {kH, kI, 2, kS};
+  const uint64_t sGu[3] = {kH * 2, (uint64_t)kI * kH * 2, estride};
+  const uint32_t bGu[4] = {kBK, kBM, 2, 1};
+  // down as (k, row, expert): one box = 256 rows, two M tiles
   const uint64_t dDn[3] = {kI, kH, kE}, dDnS[3] = {kI, kH, kS}, sDn[2] = {kI * 2, estride};
-  const uint32_t bA[3] = {kBK, kBM, 1};
+  const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
   const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
   const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
   const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
   const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
   const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, kBoxRows)};
-  if (make_map(&mGuR, expert_w, 3, dGu, sGu, bA) || make_map(&mGuS, shared_w, 3, dGuS, sGu, bA) ||
-      make_map(&mDnR, dr, 3, dDn, sDn, bA) || make_map(&mDnS, dsh, 3, dDnS, sDn, bA) ||
+  if (make_map(&mGuR, expert_w, 4, dGu, sGu, bGu) || make_map(&mGuS, shared_w, 4, dGuS, sGu, bGu) ||
+      make_map(&mDnR, dr, 3, dDn, sDn, bDn) || make_map(&mDnS, dsh, 3, dDnS, sDn, bDn) ||
       make_map(&mXr, b.xperm, 2, dXr, sX, bXr) || make_map(&mXs, x, 2, dXs, sX, bXs) ||
       make_map(&mAct, b.act, 2, dAct, sAct, bAct))
     return VG_ERR_CUDA;
@@ -353,10 +357,9 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   a.E = kE;
   a.S = kS;
   a.mblk_gu = kI / kBM;
-  a.mblk_dn = kH / kBM;
+  a.mblk_dn = kH / (2 * kBM);
   a.kc_gu = kH / kBK;
   a.kc_dn = kI / kBK;
-  a.a_up_row = kI;
   a.box_xr = (int)bXr[1];
   a.box_xs = (int)bXs[1];
   a.box_act = (int)bAct[1];
