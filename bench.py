@@ -64,6 +64,120 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _bf16_peak():
+    """Dense bf16 TFLOP/s for a kernel timed alone (the burst figure)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+PREFILL_T = 32 * 1156  # 32 pages x 1,156 visual tokens
+# FLOP of one prefill MoE layer: routed SwiGLU experts (gate, up, down) on 6T
+# rows, the two shared experts on T rows each, the router
+PREFILL_FLOP = 2 * TOPK * PREFILL_T * 3 * I * H + 2 * S * PREFILL_T * 3 * I * H + 2 * PREFILL_T * E * H
+
+
+def measure_prefill(vgv, si, dev, reps=10):
+    """One MoE layer at the prefill shape (T = 36,992, near-uniform routing), timed
+    with CUDA events: the whole layer and, through the timing hook, the expert
+    GEMM launch (the tensor-bound kernel)."""
+    import torch
+
+    d = si.FULL
+    lw = si.torch_layer_weights(SEED, 3, 0, d, device=dev)
+    x = si.torch_normal_bf16((PREFILL_T, H), 1.0, SEED, 3, si.TID_X, device=dev)
+    out = torch.empty_like(x)
+    ws = torch.empty(vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, PREFILL_T), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def layer():
+        vgv.vg_moe_ffn(vgv.MOE_DIMS, PREFILL_T, x, lw["router_w"], None, lw["expert_w"], lw["shared_w"], 1, out, None, ws)
+
+    for _ in range(3):
+        layer()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        layer()
+    e1.record(stream)
+    e1.synchronize()
+    layer_ms = e0.elapsed_time(e1) / reps
+    kinds = {vgv.VG_KERNEL_ROUTER: "router", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_EXPERTS: "expert_gemms",
+             vgv.VG_KERNEL_COMBINE: "combine"}
+    evs = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in kinds}
+    for e0_, e1_ in evs.values():
+        e0_.record(stream)
+        e1_.record(stream)
+    torch.cuda.synchronize()
+    for k, (e0_, e1_) in evs.items():
+        vgv.vg_profile_set_events(k, [e0_], [e1_])
+    parts = {n: [] for n in kinds.values()}
+    for _ in range(3):
+        layer()
+        torch.cuda.synchronize()
+        for k, (e0_, e1_) in evs.items():
+            parts[kinds[k]].append(e0_.elapsed_time(e1_))
+    for k in kinds:
+        vgv.vg_profile_set_events(k, [], [])
+    gemm = parts["expert_gemms"]
+    gemm_ms = min(gemm)
+    peak, kind = _bf16_peak()
+    gemm_flop = PREFILL_FLOP - 2 * PREFILL_T * E * H
+    del ws
+    return {"workload": f"one MoE layer, T={PREFILL_T} (32 pages x 1,156 tokens), near-uniform routing",
+            "layer_ms": layer_ms, "layer_tflops": PREFILL_FLOP / (layer_ms / 1e3) / 1e12,
+            "expert_gemms_ms": gemm_ms, "expert_gemms_tflops": gemm_flop / (gemm_ms / 1e3) / 1e12,
+            "peak_tflops": peak, "peak_source": f"{kind} bf16_tflops (burst)",
+            "frac_layer": PREFILL_FLOP / (layer_ms / 1e3) / 1e12 / peak,
+            "frac_expert_gemms": gemm_flop / (gemm_ms / 1e3) / 1e12 / peak,
+            "breakdown_ms": {n: min(v) for n, v in parts.items()}}
+
+
+def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
+    """Batch-1 verify step latency (1 sequence, K = 3 and K = 1): 12 MoE layers,
+    LM-head argmax and accept, replayed from a CUDA graph."""
+    import torch
+
+    res = {}
+    stream = torch.cuda.current_stream()
+    for k in (3, 1):
+        t = k + 1
+        xk = x[:t].contiguous()
+        hid = torch.empty(t, H, dtype=torch.bfloat16, device=dev)
+        dr = torch.zeros(1, k, dtype=torch.int32, device=dev)
+        am = torch.empty(t, dtype=torch.int32, device=dev)
+        ac = torch.empty(1, dtype=torch.int32, device=dev)
+        tk = torch.empty(1, k + 1, dtype=torch.int32, device=dev)
+        ws_s = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, t), dtype=torch.uint8, device=dev)
+        ws_v = torch.empty(vgv.vg_verify_workspace_bytes(1, k, H, V), dtype=torch.uint8, device=dev)
+
+        def step():
+            vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, t, xk, rw, None, ew, sw, hid, ws_s)
+            vgv.vg_verify_greedy(1, k, H, V, hid, lm, dr, am, ac, tk, ws_v)
+
+        step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        res[f"K{k}_ms_per_step"] = e0.elapsed_time(e1) / reps
+        del g
+    res["workload"] = "B=1 verify step (K=3: 4 tokens, K=1: 2 tokens), 12 layers + LM head + accept, CUDA graph"
+    return res
+
+
 def _cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -348,6 +462,10 @@ def run_gpu(args, rank, world, local):
     achieved = gu_bytes / (sum(gu) / 1e3) / 1e9
     launches_per_step = sum(counts.values())
 
+    # ---- the other shapes of the workload, measured on their own (untimed by the step)
+    prefill = measure_prefill(vgv, si, dev) if not args.no_extra else None
+    latency = measure_latency(vgv, x, rw, ew, sw, lm, dev) if not args.no_extra else None
+
     # ---- aggregate over ranks (max time, summed tokens)
     if world > 1:
         t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
@@ -382,6 +500,8 @@ def run_gpu(args, rank, world, local):
         "breakdown_ms_per_step": breakdown,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "prefill": prefill,
+        "batch1_latency": latency,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -399,6 +519,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["vgv", "reference"], default="vgv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the prefill and batch-1 measurements")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = _env()

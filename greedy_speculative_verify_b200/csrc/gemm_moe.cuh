@@ -226,7 +226,9 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      const uint64_t pol_w = policy_evict_first();
+      // decode tiles read an expert's weights once: stream them past L2; prefill
+      // tiles re-read them once per token tile, so they stay at normal priority
+      const uint64_t pol_w = NMAX == 64 ? policy_evict_first() : policy_evict_normal();
       int stage = 0, slot = 0;
       uint32_t phase = 0, rphase = 0, issued = 0, last_par = 0;
       auto next_stage = [&]() {

@@ -110,14 +110,27 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
     for (int j = 0; j < 4; ++j) acc[i][j] = q01[i][j] = q2[i][j] = 0.0f;
   const int HQ = H / 4;
 
+  // the next chunk's x and w are loaded into registers while the current one
+  // is multiplied, so the loads never stall the fma loop
+  uint4 xv[2], wv;
+  auto load_chunk = [&](int k0) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int q = tid + r * 256;
+      const int tok = q >> 2, kq = (q & 3) * 8;
+      xv[r] = make_uint4(0, 0, 0, 0);
+      if (t0 + tok < T) xv[r] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tok) * H + k0 + kq));
+    }
+    wv = __ldg(reinterpret_cast<const uint4*>(w + (size_t)(tid >> 2) * H + k0 + (tid & 3) * 8));
+  };
+  load_chunk(0);
   for (int k0 = 0; k0 < H; k0 += BK) {
     // x tile: 128 tokens x 32 k = 512 uint4
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int q = tid + r * 256;
       const int tok = q >> 2, kq = (q & 3) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t0 + tok < T) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tok) * H + k0 + kq));
+      const uint4 v = xv[r];
       xs[(kq + 0) * XS + tok] = bf16_lo(v.x);
       xs[(kq + 1) * XS + tok] = bf16_hi(v.x);
       xs[(kq + 2) * XS + tok] = bf16_lo(v.y);
@@ -129,7 +142,7 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
     }
     {
       const int ex = tid >> 2, kq = (tid & 3) * 8;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(w + (size_t)ex * H + k0 + kq));
+      const uint4 v = wv;
       ws[(kq + 0) * WS + ex] = bf16_lo(v.x);
       ws[(kq + 1) * WS + ex] = bf16_hi(v.x);
       ws[(kq + 2) * WS + ex] = bf16_lo(v.y);
@@ -139,6 +152,7 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
       ws[(kq + 6) * WS + ex] = bf16_lo(v.w);
       ws[(kq + 7) * WS + ex] = bf16_hi(v.w);
     }
+    if (k0 + BK < H) load_chunk(k0 + BK);
     __syncthreads();
 #pragma unroll 8
     for (int kk = 0; kk < BK; ++kk) {
