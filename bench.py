@@ -49,6 +49,10 @@ WORKLOAD = {
     "l2": "inputs larger than L2: 5.78 GB of weights per step vs 126 MB L2, no flush",
 }
 EXPERT_W_BYTES = 3 * I * H * 2  # gate + up + down of one expert, bf16 (6,881,280 B)
+# DRAM bytes (read + write) of one expert-GEMM launch at 128 tokens, from one
+# ncu capture of that kernel (456.5 MB read + 5.1 MB written); to be re-taken
+# whenever that kernel changes
+EXPERT_TRAFFIC_BYTES = 461.6e6
 
 
 def _env():
@@ -494,7 +498,7 @@ def run_gpu(args, rank, world, local):
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "kernel": "moe_expert_gemms (gate/up + SwiGLU + down, routed + shared)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": EXPERT_TRAFFIC_BYTES,
                      "algorithmic_bytes_per_launch": gu_bytes / max(1, len(gu)),
                      "avg_launch_ms": sum(gu) / max(1, len(gu))},
         "breakdown_ms_per_step": breakdown,
