@@ -47,13 +47,15 @@ constexpr int kNMax = 128;     // tokens per tile, widest configuration
 constexpr int kBoxRows = 32;   // token rows per TMA box of the B operand
 constexpr int kMaxExperts = 72;
 
-// Two configurations of the same kernel, by tile width NMAX:
+// Three configurations of the same kernel, by tile width NMAX:
 //  * NMAX = 128, 4 stages: prefill-sized expert segments, 128 x 128 tiles;
 //  * NMAX = 64, 5 stages: decode sizes, where the token slot of a stage is
-//    small and the freed shared memory buys a fifth stage of weights in flight.
+//    small and the freed shared memory buys a fifth stage of weights in flight;
+//  * NMAX = 16, 6 stages: a handful of tokens (batch-1 verify), where every
+//    expert's tokens fit one 16-row tile and a sixth stage fits.
 template <int NMAX>
 struct FgCfg {
-  static constexpr int kStages = NMAX == 128 ? 4 : 5;
+  static constexpr int kStages = NMAX == 128 ? 4 : NMAX == 64 ? 5 : 6;
   static constexpr int kABytes = 2 * kBM * kBK * 2;      // two 16 KB weight tiles
   static constexpr int kBBytes = NMAX * kBK * 2;         // token slot
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(192, 1)
       // ------------------------------------------------------------ producer
       // decode tiles read an expert's weights once: stream them past L2; prefill
       // tiles re-read them once per token tile, so they stay at normal priority
-      const uint64_t pol_w = NMAX == 64 ? policy_evict_first() : policy_evict_normal();
+      const uint64_t pol_w = NMAX <= 64 ? policy_evict_first() : policy_evict_normal();
       int stage = 0, slot = 0;
       uint32_t phase = 0, rphase = 0, issued = 0, last_par = 0;
       auto next_stage = [&]() {

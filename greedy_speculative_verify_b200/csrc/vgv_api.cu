@@ -87,7 +87,9 @@ vg_status device_state(DevState** out) {
     if (cudaFuncSetAttribute(vg::moe_expert_gemms<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::FgCfg<128>::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vg::moe_expert_gemms<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vg::FgCfg<64>::kSmemBytes) != cudaSuccess)
+                             vg::FgCfg<64>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vg::moe_expert_gemms<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::FgCfg<16>::kSmemBytes) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::moe_layer_entry<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::layer_entry_smem()) != cudaSuccess)
@@ -136,13 +138,17 @@ struct MoeWs {
   int sched_len;
 };
 
-// Upper bound of the expert GEMMs' token tiles: routed segments cut at 128 plus
-// one partial tile per routed expert, plus the shared experts' tiles.
-int max_tiles(int T) { return vg::cdiv(T * kTopK, 64) + kE + kS * vg::cdiv(T, 64); }
+// Tile width of the expert GEMMs: 16-token tiles (six pipeline stages) for a
+// handful of tokens, 64-token tiles (five stages) at decode sizes, 128-token
+// tiles for prefill-sized segments.
+int expert_tile(int T) { return T <= 16 ? 16 : T <= 1024 ? 64 : 128; }
 
-// Tile width of the expert GEMMs: 64-token tiles (and a fifth pipeline stage)
-// at decode sizes, 128-token tiles for prefill-sized segments.
-int expert_tile(int T) { return T <= 1024 ? 64 : 128; }
+// Upper bound of the expert GEMMs' token tiles: routed segments cut at the tile
+// width plus one partial tile per routed expert, plus the shared experts' tiles.
+int max_tiles(int T) {
+  const int nt = expert_tile(T);
+  return vg::cdiv(T * kTopK, nt) + kE + kS * vg::cdiv(T, nt);
+}
 
 MoeWs moe_layout(int T) {
   const size_t N = (size_t)T * kTopK;
@@ -233,6 +239,7 @@ struct PrevCombine {
 // of the first routed experts, which the expert kernel's first wave of units
 // streams (about one unit per SM).
 constexpr size_t kEntryPrefetchBytes = (size_t)96 << 20;
+constexpr int kEntryPrefetchMinT = 64;  // 384 assignments: each expert untouched with probability < 0.3%
 
 // Launch of a decode-path kernel with programmatic stream serialization (the
 // kernel waits for its predecessor itself, see griddep_wait), optionally
@@ -288,7 +295,9 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     a.gbar_base = *nbar;
     const size_t gu_bytes = (size_t)2 * kI * kH * 2;
     a.prefetch_base = static_cast<const uint8_t*>(expert_w);
-    a.n_prefetch = (int)min((size_t)kE, kEntryPrefetchBytes / gu_bytes);
+    // only when nearly every expert is touched: otherwise most of the prefetched
+    // bytes would belong to experts no token chose
+    a.n_prefetch = T >= kEntryPrefetchMinT ? (int)min((size_t)kE, kEntryPrefetchBytes / gu_bytes) : 0;
     a.prefetch_bytes = (uint32_t)gu_bytes;
     a.prefetch_stride = (uint64_t)3 * kI * kH * 2;
     const int grid = entry_grid(dev, T);
@@ -343,9 +352,10 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
   const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
   const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
-  const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, kBoxRows)};
-  const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, kBoxRows)};
-  const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, kBoxRows)};
+  const int nt = expert_tile(T), bx = std::min(kBoxRows, nt);  // a box never exceeds the token slot
+  const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, bx)};
+  const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, bx)};
+  const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, bx)};
   if (make_map(&mGuR, expert_w, 4, dGu, sGu, bGu) || make_map(&mGuS, shared_w, 4, dGuS, sGu, bGu) ||
       make_map(&mDnR, dr, 3, dDn, sDn, bDn) || make_map(&mDnS, dsh, 3, dDnS, sDn, bDn) ||
       make_map(&mXr, b.xperm, 2, dXr, sX, bXr) || make_map(&mXs, x, 2, dXs, sX, bXs) ||
@@ -369,7 +379,10 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
   ProfScope ps(VG_KERNEL_EXPERTS, s);
   const cudaError_t e =
-      expert_tile(T) == 64
+      nt == 16
+          ? launch_dep(moe_expert_gemms<16>, grid, 192, FgCfg<16>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS, mXr,
+                       mXs, mAct, a)
+      : nt == 64
           ? launch_dep(moe_expert_gemms<64>, grid, 192, FgCfg<64>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS, mXr,
                        mXs, mAct, a)
           : launch_dep(moe_expert_gemms<128>, grid, 192, FgCfg<128>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS,
