@@ -28,6 +28,7 @@ EXPORTS = (
     "vg_moe_stack_workspace_bytes", "vg_moe_ffn_stack", "vg_verify_workspace_bytes",
     "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag",
     "vg_profile_set_events", "vg_profile_count", "vg_verify_greedy_noalloc",
+    "vg_embed_rows", "vg_spec_rows", "vg_spec_commit",
 )
 
 # vg_kernel
@@ -50,6 +51,14 @@ class vg_moe_taps(ctypes.Structure):
     _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_weight", ctypes.c_void_p),
                 ("expert_offsets", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("inv_perm", ctypes.c_void_p),
                 ("act", ctypes.c_void_p), ("expert_out", ctypes.c_void_p)]
+
+
+class vg_spec_state(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("K", ctypes.c_int32), ("V", ctypes.c_int32),
+                ("last", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("committed", ctypes.c_void_p),
+                ("cap", ctypes.c_int32), ("ref", ctypes.c_void_p), ("ref_len", ctypes.c_int32),
+                ("p", ctypes.c_float), ("seed", ctypes.c_uint64), ("step", ctypes.c_void_p),
+                ("tokens", ctypes.c_void_p), ("drafts", ctypes.c_void_p)]
 
 
 MOE_DIMS = vg_moe_dims(1280, 896, 64, 2, 6)
@@ -83,6 +92,9 @@ def load():
         "vg_profile_set_events": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
         "vg_profile_count": (ctypes.c_int64, [i32]),
         "vg_verify_greedy_noalloc": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+        "vg_embed_rows": (i32, [vp, i32, vp, i32, i32, vp, vp]),
+        "vg_spec_rows": (i32, [ctypes.POINTER(vg_spec_state), vp]),
+        "vg_spec_commit": (i32, [ctypes.POINTER(vg_spec_state), vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -205,3 +217,31 @@ def vg_verify_greedy_noalloc(B, K, H, V, h, lm_head, drafts, argmax, accepted, o
     st = load().vg_verify_greedy_noalloc(B, K, H, V, _ptr(h), _ptr(lm_head), _ptr(drafts), _ptr(argmax),
                                          _ptr(accepted), _ptr(out_tokens), _stream(stream))
     _check(st, "vg_verify_greedy_noalloc")
+
+
+# ------------------------------------------------------------ decode loop
+def vg_embed_rows(tokens, emb, out, stream=None):
+    """out[i] = emb[tokens[i]] (bf16 rows)."""
+    _check(load().vg_embed_rows(_ptr(tokens), tokens.numel(), _ptr(emb), emb.shape[0], emb.shape[1], _ptr(out),
+                                _stream(stream)), "vg_embed_rows")
+
+
+def make_spec_state(B, K, V, last, pos, committed, ref, p, seed, step, tokens, drafts):
+    """vg_spec_state over caller-owned device tensors (ref may be None); every
+    tensor is read as dense rows, so each must be contiguous."""
+    for t in (last, pos, committed, ref, step, tokens, drafts):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("vg_spec_state tensors must be contiguous")
+    return vg_spec_state(B, K, V, last.data_ptr(), pos.data_ptr(), committed.data_ptr(), committed.shape[1],
+                         None if ref is None else ref.data_ptr(), 0 if ref is None else ref.shape[1],
+                         float(p), int(seed), step.data_ptr(), tokens.data_ptr(),
+                         None if drafts is None else drafts.data_ptr())
+
+
+def vg_spec_rows(state, stream=None):
+    _check(load().vg_spec_rows(ctypes.byref(state), _stream(stream)), "vg_spec_rows")
+
+
+def vg_spec_commit(state, accepted, out_tokens, stream=None):
+    _check(load().vg_spec_commit(ctypes.byref(state), _ptr(accepted), _ptr(out_tokens), _stream(stream)),
+           "vg_spec_commit")

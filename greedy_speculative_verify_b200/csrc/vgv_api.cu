@@ -11,6 +11,7 @@
 #include "vgv.h"
 #include "common.cuh"
 #include "combine.cuh"
+#include "decode_loop.cuh"
 #include "gemm_moe.cuh"
 #include "layer_entry.cuh"
 #include "lmhead.cuh"
@@ -242,10 +243,11 @@ constexpr size_t kEntryPrefetchBytes = (size_t)96 << 20;
 constexpr int kEntryPrefetchMinT = 64;  // 384 assignments: each expert untouched with probability < 0.3%
 
 // Launch of a decode-path kernel with programmatic stream serialization (the
-// kernel waits for its predecessor itself, see griddep_wait), optionally
+// kernel waits for its predecessor itself, see griddep_wait), plain or
 // cooperative.
+enum class Launch { kPlain, kCooperative };  // a distinct type: no argument converts to it by accident
 template <typename... KArgs, typename... Args>
-cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, bool coop,
+cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Launch kind,
                        Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -258,7 +260,7 @@ cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, size_t smem,
   attr[1].id = cudaLaunchAttributeCooperative;
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = coop ? 2 : 1;
+  cfg.numAttrs = kind == Launch::kCooperative ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -307,7 +309,7 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     const uint32_t bR[2] = {64, kE};
     if (make_map(&mR, router_w, 2, dR, sR, bR)) return VG_ERR_CUDA;
     ProfScope ps(VG_KERNEL_ROUTER, s);
-    if (launch_dep(moe_layer_entry<kTopK>, grid, kEntryThreads, layer_entry_smem(), s, true, mR, a) != cudaSuccess)
+    if (launch_dep(moe_layer_entry<kTopK>, grid, kEntryThreads, layer_entry_smem(), s, Launch::kCooperative, mR, a) != cudaSuccess)
       return cuda_fail();
     return VG_OK;
   }
@@ -380,12 +382,12 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   ProfScope ps(VG_KERNEL_EXPERTS, s);
   const cudaError_t e =
       nt == 16
-          ? launch_dep(moe_expert_gemms<16>, grid, 192, FgCfg<16>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS, mXr,
+          ? launch_dep(moe_expert_gemms<16>, grid, 192, FgCfg<16>::kSmemBytes, s, Launch::kPlain, mGuR, mGuS, mDnR, mDnS, mXr,
                        mXs, mAct, a)
       : nt == 64
-          ? launch_dep(moe_expert_gemms<64>, grid, 192, FgCfg<64>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS, mXr,
+          ? launch_dep(moe_expert_gemms<64>, grid, 192, FgCfg<64>::kSmemBytes, s, Launch::kPlain, mGuR, mGuS, mDnR, mDnS, mXr,
                        mXs, mAct, a)
-          : launch_dep(moe_expert_gemms<128>, grid, 192, FgCfg<128>::kSmemBytes, s, false, mGuR, mGuS, mDnR, mDnS,
+          : launch_dep(moe_expert_gemms<128>, grid, 192, FgCfg<128>::kSmemBytes, s, Launch::kPlain, mGuR, mGuS, mDnR, mDnS,
                        mXr, mXs, mAct, a);
   return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
 }
@@ -393,7 +395,7 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
 vg_status launch_combine(int T, const void* x, const LayerBufs& b, int add_residual, void* out, cudaStream_t s) {
   using namespace vg;
   ProfScope ps(VG_KERNEL_COMBINE, s);
-  const cudaError_t e = launch_dep(moe_combine, cdiv(T * (kH / 8), 256), 256, 0, s, false,
+  const cudaError_t e = launch_dep(moe_combine, cdiv(T * (kH / 8), 256), 256, 0, s, Launch::kPlain,
                                    static_cast<const __nv_bfloat16*>(x), (const __nv_bfloat16*)b.o,
                                    (const int32_t*)b.inv, (const float*)b.gw, T, kH, kTopK, kS, add_residual,
                                    static_cast<__nv_bfloat16*>(out));
@@ -563,14 +565,14 @@ vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V, const voi
   const int grid = min(dev->sms, n_mblk * n_groups);
   {
   ProfScope ps(VG_KERNEL_LM_HEAD, s);
-  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, false, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
+  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, Launch::kPlain, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
                  kLmGroupTiles, n_groups, a_box_rows, box_rows(V, kLmN), part) != cudaSuccess)
     return VG_ERR_CUDA;
   }
   const int spb = max(1, 32 / (K + 1));
   {
     ProfScope ps(VG_KERNEL_ACCEPT, s);
-    if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, false, (const uint64_t*)part, n_groups, R, B, K, drafts,
+    if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, Launch::kPlain, (const uint64_t*)part, n_groups, R, B, K, drafts,
                    argmax, accepted, out_tokens) != cudaSuccess)
       return VG_ERR_CUDA;
   }
@@ -693,12 +695,73 @@ extern "C" vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, i
     if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
   }
   const int grid = min(dev->sms, n_mblk * n_groups);
-  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, false, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
+  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, Launch::kPlain, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
                  kLmGroupTiles, n_groups, a_box_rows, box_rows(V, kLmN), part) != cudaSuccess)
     return VG_ERR_CUDA;
   const int spb = max(1, 32 / (K + 1));
-  if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, false, (const uint64_t*)part, n_groups, R, B, K, drafts,
+  if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, Launch::kPlain, (const uint64_t*)part, n_groups, R, B, K, drafts,
                  argmax, accepted, out_tokens) != cudaSuccess)
     return VG_ERR_CUDA;
   return VG_OK;
+}
+
+// ------------------------------------------------------------ decode loop
+namespace {
+bool spec_state_ok(const vg_spec_state* st) {
+  if (st == nullptr || st->B < 0 || st->K < 0 || st->K > 64 || st->V <= 0 || st->cap < 0 || st->ref_len < 0)
+    return false;
+  if (!(st->p >= 0.0f && st->p <= 1.0f)) return false;
+  if (st->B == 0) return true;
+  if (!st->last || !st->pos || !st->step || !st->tokens || (st->cap > 0 && !st->committed)) return false;
+  if (st->K > 0 && !st->drafts) return false;
+  if (st->ref_len > 0 && !st->ref) return false;
+  return true;
+}
+vg::SpecState spec_dev(const vg_spec_state* st) {
+  vg::SpecState s{};
+  s.B = st->B;
+  s.K = st->K;
+  s.V = st->V;
+  s.last = st->last;
+  s.pos = st->pos;
+  s.committed = st->committed;
+  s.cap = st->cap;
+  s.ref = st->ref;
+  s.ref_len = st->ref_len;
+  s.p = st->p;
+  s.seed = st->seed;
+  s.step = st->step;
+  s.tokens = st->tokens;
+  s.drafts = st->drafts;
+  return s;
+}
+}  // namespace
+
+extern "C" vg_status vg_embed_rows(const int32_t* tokens, int32_t n, const void* emb, int32_t V, int32_t H, void* out,
+                                   vg_stream_t stream) {
+  if (n < 0 || V <= 0 || H <= 0 || H % 8 != 0) return VG_ERR_INVALID_ARG;
+  if (n == 0) return VG_OK;
+  if (!tokens || !emb || !out || !aligned16(emb) || !aligned16(out)) return VG_ERR_INVALID_ARG;
+  if (overlaps(emb, (size_t)V * H * 2, out, (size_t)n * H * 2)) return VG_ERR_INVALID_ARG;
+  const cudaError_t e = launch_dep(vg::embed_rows, vg::cdiv(n, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream), Launch::kPlain,
+                                   tokens, (int)n, static_cast<const __nv_bfloat16*>(emb), (int)V, (int)H,
+                                   static_cast<__nv_bfloat16*>(out));
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+extern "C" vg_status vg_spec_rows(const vg_spec_state* st, vg_stream_t stream) {
+  if (!spec_state_ok(st)) return VG_ERR_INVALID_ARG;
+  if (st->B == 0) return VG_OK;
+  const cudaError_t e = launch_dep(vg::spec_rows, vg::cdiv(st->B, 128), 128, 0, reinterpret_cast<cudaStream_t>(stream),
+                                   Launch::kPlain, spec_dev(st));
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+extern "C" vg_status vg_spec_commit(const vg_spec_state* st, const int32_t* accepted, const int32_t* out_tokens,
+                                    vg_stream_t stream) {
+  if (!spec_state_ok(st) || (st->B > 0 && (!accepted || !out_tokens))) return VG_ERR_INVALID_ARG;
+  if (st->B == 0) return VG_OK;
+  const cudaError_t e = launch_dep(vg::spec_commit, vg::cdiv(st->B, 128), 128, 0,
+                                   reinterpret_cast<cudaStream_t>(stream), Launch::kPlain, spec_dev(st), accepted, out_tokens);
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
 }

@@ -235,6 +235,66 @@ vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, int32_t V,
                                    int32_t* argmax, int32_t* accepted, int32_t* out_tokens,
                                    vg_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Multi-step speculative decoding on a synthetic Markov decoder (device-side
+ * bookkeeping between verify steps). The pages verify K drafted tokens per
+ * step and commit the longest prefix on which draft and verifier agree plus
+ * the verifier's own token, so the committed text equals plain greedy decoding
+ * ("jina-ocr-v1: Schnellere Dokumentenanalyse auf kostengünstigen GPUs",
+ * "Modell und Training"; "Jina AI's 3.4B OCR model targets faster page
+ * parsing", "FastMTP cuts decoding work"). These calls let a loop of
+ *   vg_spec_rows -> vg_embed_rows -> vg_moe_ffn_stack -> vg_verify_greedy ->
+ *   vg_spec_commit
+ * run step after step on the device (and be captured in one CUDA graph), for a
+ * decoder whose next token is argmax(LM head(MoE stack(emb[last token]))). The
+ * draft source is synthetic: the decoder's own token from a reference
+ * continuation with probability p, else a uniform token (the pages' drafter is
+ * a trained block that is not on this path). K = 0 is plain greedy decoding.
+ * ------------------------------------------------------------------------- */
+
+/* out[i, :] = emb[tokens[i], :] for i < n. tokens int32 [n]; emb bf16 [V, H];
+ * out bf16 [n, H]; H a multiple of 8, 16-byte aligned rows. A token outside
+ * [0, V) gives a zero row and records VG_ERR_DEVICE_BOUNDS in the status word.
+ * Errors: VG_ERR_INVALID_ARG, VG_ERR_CUDA. */
+vg_status vg_embed_rows(const int32_t* tokens, int32_t n, const void* emb, int32_t V, int32_t H, void* out,
+                        vg_stream_t stream);
+
+/* State of B sequences being decoded, all in device memory and owned by the
+ * caller. last[b] starts as the prompt's last token, pos[b] as 0, *step as 0.
+ * committed [B, cap] receives the committed tokens (positions >= cap are
+ * counted in pos but not stored). ref [B, ref_len]: the reference continuation
+ * (ref[b, j] = the token greedy decoding commits at position j), read only by
+ * the draft source. Random draws: SplitMix64 on a counter of (seed, step, b,
+ * draft index). */
+typedef struct vg_spec_state {
+  int32_t B, K, V;
+  int32_t* last;        /* [B] */
+  int32_t* pos;         /* [B] */
+  int32_t* committed;   /* [B, cap] */
+  int32_t cap;
+  const int32_t* ref;   /* [B, ref_len] or NULL with ref_len = 0 (uniform drafts only) */
+  int32_t ref_len;
+  float p;              /* probability that a draft is the reference token, in [0, 1] */
+  uint64_t seed;
+  int32_t* step;        /* [1] steps taken, advanced by vg_spec_commit */
+  int32_t* tokens;      /* [B, K+1] the next verify rows: last token, then the drafts */
+  int32_t* drafts;      /* [B, K] the drafts alone (the verify call's input) */
+} vg_spec_state;
+
+/* Writes the next verify rows (tokens) and drafts of every sequence: draft i
+ * (1..K) is ref[b, pos[b] + i - 1] with probability p (if that position is
+ * below ref_len), else a uniform token in [0, V). Errors: VG_ERR_INVALID_ARG,
+ * VG_ERR_CUDA. */
+vg_status vg_spec_rows(const vg_spec_state* st, vg_stream_t stream);
+
+/* After vg_verify_greedy on those rows: appends out_tokens[b, 0..accepted[b]]
+ * to committed at pos[b], advances pos[b] by accepted[b] + 1, sets last[b] to
+ * the bonus token and advances *step. accepted int32 [B] in [0, K] (others
+ * record VG_ERR_DEVICE_BOUNDS and count as 0); out_tokens int32 [B, K+1].
+ * Errors: VG_ERR_INVALID_ARG, VG_ERR_CUDA. */
+vg_status vg_spec_commit(const vg_spec_state* st, const int32_t* accepted, const int32_t* out_tokens,
+                         vg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

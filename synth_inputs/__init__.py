@@ -39,6 +39,7 @@ TID_SHARED = 3
 TID_LM_HEAD = 4
 TID_DRAFTS = 5
 TID_HID = 6
+TID_EMB = 7  # token embedding of the synthetic decoder
 
 
 @dataclasses.dataclass(frozen=True)

@@ -116,3 +116,25 @@ def test_binding_has_no_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(vgv, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         vgv.vg_abi_version()
+
+
+def test_decode_loop_validation_before_launch(lib):
+    A = 1 << 40
+    # embedding gather: bad sizes, null pointers, misaligned rows
+    assert lib.vg_embed_rows(A, 0, A, 10, 1280, A + (1 << 30), None) == 0          # n = 0: no-op
+    assert lib.vg_embed_rows(A, -1, A, 10, 1280, A + (1 << 30), None) == 1
+    assert lib.vg_embed_rows(A, 4, A, 10, 1281, A + (1 << 30), None) == 1          # H not a multiple of 8
+    assert lib.vg_embed_rows(None, 4, A, 10, 1280, A + (1 << 30), None) == 1
+    assert lib.vg_embed_rows(A, 4, A + 8, 10, 1280, A + (1 << 30), None) == 1      # misaligned table
+    assert lib.vg_embed_rows(A, 4, A, 10, 1280, A + 64, None) == 1                 # out overlaps the table
+    # speculative-loop state
+    mk = lambda **kw: vgv.vg_spec_state(**{**dict(B=2, K=3, V=100, last=A, pos=A, committed=A, cap=8, ref=None,
+                                                  ref_len=0, p=0.5, seed=1, step=A, tokens=A, drafts=A), **kw})
+    f_rows, f_commit = lib.vg_spec_rows, lib.vg_spec_commit
+    assert f_rows(None, None) == 1
+    assert f_rows(ctypes.byref(mk(p=1.5)), None) == 1
+    assert f_rows(ctypes.byref(mk(K=3, drafts=None)), None) == 1                   # drafts needed for K > 0
+    assert f_rows(ctypes.byref(mk(ref_len=4)), None) == 1                          # ref_len without ref
+    assert f_rows(ctypes.byref(mk(B=0)), None) == 0                                # B = 0: no-op
+    assert f_commit(ctypes.byref(mk()), None, A, None) == 1                        # accepted needed
+    assert f_commit(ctypes.byref(mk(B=0)), None, None, None) == 0
