@@ -140,6 +140,78 @@ def measure_prefill(vgv, si, dev, reps=10):
             "breakdown_ms": {n: min(v) for n, v in parts.items()}}
 
 
+def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
+    """Multi-step speculative decoding of B=32 sequences at K=3 on the device,
+    on a synthetic Markov decoder (embedding of the last token -> the 12 MoE
+    layers -> LM head -> argmax): one step = draft rows, embedding gather,
+    layer stack, verify, commit, replayed from a CUDA graph. Drafts are the
+    decoder's own token (from a plain greedy run of the same loop) with
+    probability p, else uniform. Reports committed tokens/s, tau, and whether
+    the committed tokens equal the greedy run's."""
+    import torch
+
+    i32 = dict(dtype=torch.int32, device=dev)
+    emb = si.torch_normal_bf16((V, H), 1.0, SEED, CFG, si.TID_EMB, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(SEED + 23)
+    starts = torch.randint(0, V, (B,), generator=g, device=dev, dtype=torch.int32)
+    stream = torch.cuda.current_stream()
+
+    def loop(K, n_tokens, ref=None, steps=None):
+        T_ = B * (K + 1)
+        last, pos, step = starts.clone(), torch.zeros(B, **i32), torch.zeros(1, **i32)
+        cap = n_tokens + (K + 1) * ((steps or 0) + 5) + K + 1  # every step of the run fits
+        committed = torch.full((B, cap), -1, **i32)
+        tokens, drafts = torch.empty(B, K + 1, **i32), torch.empty(B, max(K, 1), **i32)
+        x = torch.empty(T_, H, dtype=torch.bfloat16, device=dev)
+        hid = torch.empty_like(x)
+        am, acc, out = torch.empty(T_, **i32), torch.empty(B, **i32), torch.empty(B, K + 1, **i32)
+        ws_s = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, T_), dtype=torch.uint8, device=dev)
+        ws_v = torch.empty(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
+        st = vgv.make_spec_state(B, K, V, last, pos, committed, ref, p, SEED + 29, step, tokens, drafts if K else None)
+
+        def one():
+            vgv.vg_spec_rows(st)
+            vgv.vg_embed_rows(tokens.view(-1), emb, x)
+            vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, T_, x, rw, None, ew, sw, hid, ws_s)
+            vgv.vg_verify_greedy(B, K, H, V, hid, lm, drafts if K else None, am, acc, out, ws_v)
+            vgv.vg_spec_commit(st, acc, out)
+
+        one()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            one()
+        if steps is None:  # run until every sequence has n_tokens
+            while int(pos.min()) < n_tokens:
+                gr.replay()
+            torch.cuda.synchronize()
+            return committed, None, None
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        p0 = int(pos.sum())
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            gr.replay()
+        e1.record(stream)
+        e1.synchronize()
+        return committed, int(pos.sum()) - p0, e0.elapsed_time(e1) / steps
+
+    ref_len = (n_steps + 5) * (K + 1) + K + 1
+    greedy, _, _ = loop(0, ref_len)
+    greedy = greedy[:, :ref_len].contiguous()
+    spec, tokens_timed, ms = loop(K, 0, ref=greedy, steps=n_steps)
+    n_cmp = min(int((spec >= 0).sum(1).min()), ref_len)
+    lossless = bool(torch.equal(spec[:, :n_cmp], greedy[:, :n_cmp]))
+    return {"workload": f"B={B} sequences, K={K}, {LAYERS} layers, V={V}: device loop of draft rows, embedding, "
+                        f"MoE stack, verify, commit (CUDA graph), {n_steps} timed steps",
+            "tokens_per_s": tokens_timed / (ms * n_steps / 1e3), "ms_per_step": ms,
+            "tau": tokens_timed / (B * n_steps), "draft_p": p,
+            "lossless_vs_greedy": lossless, "tokens_compared": n_cmp * B}
+
+
 def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
     """Batch-1 verify step latency (1 sequence, K = 3 and K = 1): 12 MoE layers,
     LM-head argmax and accept, replayed from a CUDA graph."""
@@ -469,6 +541,7 @@ def run_gpu(args, rank, world, local):
     # ---- the other shapes of the workload, measured on their own (untimed by the step)
     prefill = measure_prefill(vgv, si, dev) if not args.no_extra else None
     latency = measure_latency(vgv, x, rw, ew, sw, lm, dev) if not args.no_extra else None
+    spec_loop = measure_spec_loop(vgv, si, rw, ew, sw, lm, dev) if not args.no_extra else None
 
     # ---- aggregate over ranks (max time, summed tokens)
     if world > 1:
@@ -506,6 +579,7 @@ def run_gpu(args, rank, world, local):
         "cpu_baseline": cpu,
         "prefill": prefill,
         "batch1_latency": latency,
+        "spec_decode_loop": spec_loop,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
