@@ -323,6 +323,22 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ GPU leg
 
+def aggregate_over_ranks(ms, e2e_ms, tokens_rank, world, device):
+    """The job's step times are its slowest rank's (max over ranks); its
+    committed tokens are all ranks' (sum). Every rank calls this once, in the
+    same order, with the process group already initialised when world > 1."""
+    if world == 1:
+        return ms, e2e_ms, tokens_rank
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    n = torch.tensor([tokens_rank], dtype=torch.int64, device=device)
+    dist.all_reduce(n)
+    return float(t[0]), float(t[1]), int(n.item())
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons every 200 ms."""
 
@@ -544,15 +560,7 @@ def run_gpu(args, rank, world, local):
     spec_loop = measure_spec_loop(vgv, si, rw, ew, sw, lm, dev) if not args.no_extra else None
 
     # ---- aggregate over ranks (max time, summed tokens)
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-        n = torch.tensor([tokens_rank], dtype=torch.int64, device=dev)
-        dist.all_reduce(n)
-        tokens_all = int(n.item())
-    else:
-        tokens_all = tokens_rank
+    ms, e2e_ms, tokens_all = aggregate_over_ranks(ms, e2e_ms, tokens_rank, world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
