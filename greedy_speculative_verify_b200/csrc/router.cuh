@@ -87,9 +87,12 @@ constexpr int kRtPad = 8;       // elements of padding per quarter row: conflict
 
 // Large token counts: a 128-token x 64-expert block tile, staged through shared
 // memory 32 k at a time; each thread owns 8 tokens x 4 experts and runs every
-// output's chain in increasing k.
+// output's chain in increasing k. The finished quarter sums wait in (dynamic)
+// shared memory rather than registers, so that two blocks fit an SM.
+constexpr int kRtPartBytes = 2 * 128 * (kRouterE + 1) * 4;  // (q0 + q1) and q2 of a block tile
+
 template <int K>
-__global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256, 2) router_topk_tiled(const __nv_bfloat16* __restrict__ x,
                                                          const __nv_bfloat16* __restrict__ w,
                                                          const float* __restrict__ bias, int T, int H,
                                                          int32_t* __restrict__ idx_out,
@@ -101,13 +104,17 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
   const int tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;
   const int t0 = blockIdx.x * BT;
-  // quarter sums: acc runs the current quarter's chains; q01 and q2 keep the
-  // finished ones until (q0 + q1) + (q2 + q3) (H/4 is a multiple of BK)
-  float acc[8][4], q01[8][4], q2[8][4];
+  // quarter sums: acc runs the current quarter's chains; p01 and p2 keep the
+  // finished ones until (q0 + q1) + (q2 + q3) (H/4 is a multiple of BK); each
+  // thread reads back only the entries it wrote
+  extern __shared__ float rt_part[];
+  float* p01 = rt_part;               // [BT][LS]
+  float* p2 = rt_part + BT * LS;      // [BT][LS]
+  float acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = q01[i][j] = q2[i][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
   const int HQ = H / 4;
 
   // the next chunk's x and w are loaded into registers while the current one
@@ -168,19 +175,28 @@ __global__ void __launch_bounds__(256) router_topk_tiled(const __nv_bfloat16* __
     }
     __syncthreads();
     const int qend = (k0 + BK) / HQ;  // a quarter ends with this chunk when (k0 + BK) % HQ == 0
-    if ((k0 + BK) % HQ == 0) {
+    if ((k0 + BK) % HQ == 0 && qend < 4) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (qend == 1) q01[i][j] = acc[i][j];
-          else if (qend == 2) q01[i][j] = q01[i][j] + acc[i][j];
-          else if (qend == 3) q2[i][j] = acc[i][j];
-          else q01[i][j] = q01[i][j] + (q2[i][j] + acc[i][j]);
+          float* a01 = p01 + (ty * 8 + i) * LS + tx * 4 + j;
+          if (qend == 1) *a01 = acc[i][j];
+          else if (qend == 2) *a01 = *a01 + acc[i][j];
+          else p2[(ty * 8 + i) * LS + tx * 4 + j] = acc[i][j];
           acc[i][j] = 0.0f;
         }
     }
   }
+  // the last quarter ends with the last chunk: the logit is (q0 + q1) + (q2 + q3)
+  float q01[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int o = (ty * 8 + i) * LS + tx * 4 + j;
+      q01[i][j] = p01[o] + (p2[o] + acc[i][j]);
+    }
   float* logits = buf;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {

@@ -95,6 +95,9 @@ vg_status device_state(DevState** out) {
     if (cudaFuncSetAttribute(vg::moe_layer_entry<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::layer_entry_smem()) != cudaSuccess)
       return cuda_fail();
+    if (cudaFuncSetAttribute(vg::router_topk_tiled<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::kRtPartBytes) != cudaSuccess)
+      return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
       return cuda_fail();
@@ -321,8 +324,8 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
   }
   {
     ProfScope ps(VG_KERNEL_ROUTER, s);
-    router_topk_tiled<kTopK><<<cdiv(T, 128), 256, 0, s>>>(xcur, static_cast<const __nv_bfloat16*>(router_w),
-                                                         router_bias, T, kH, b.idx, b.gw);
+    router_topk_tiled<kTopK><<<cdiv(T, 128), 256, kRtPartBytes, s>>>(xcur, static_cast<const __nv_bfloat16*>(router_w),
+                                                                     router_bias, T, kH, b.idx, b.gw);
   }
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
   {
