@@ -43,7 +43,6 @@ namespace vg {
 
 constexpr int kBM = 128;       // weight rows per MMA tile
 constexpr int kBK = 64;        // K elements per stage: one 128-byte swizzle row
-constexpr int kNMax = 128;     // tokens per tile, widest configuration
 constexpr int kBoxRows = 32;   // token rows per TMA box of the B operand
 constexpr int kMaxExperts = 72;
 

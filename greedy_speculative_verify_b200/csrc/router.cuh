@@ -18,17 +18,6 @@ namespace vg {
 
 constexpr int kRouterE = 64;
 
-__device__ __forceinline__ void fma8(float& acc, uint4 a, uint4 b) {
-  acc = __fmaf_rn(bf16_lo(a.x), bf16_lo(b.x), acc);
-  acc = __fmaf_rn(bf16_hi(a.x), bf16_hi(b.x), acc);
-  acc = __fmaf_rn(bf16_lo(a.y), bf16_lo(b.y), acc);
-  acc = __fmaf_rn(bf16_hi(a.y), bf16_hi(b.y), acc);
-  acc = __fmaf_rn(bf16_lo(a.z), bf16_lo(b.z), acc);
-  acc = __fmaf_rn(bf16_hi(a.z), bf16_hi(b.z), acc);
-  acc = __fmaf_rn(bf16_lo(a.w), bf16_lo(b.w), acc);
-  acc = __fmaf_rn(bf16_hi(a.w), bf16_hi(b.w), acc);
-}
-
 // One warp selects the top-K of 64 logits of one token and writes the expert
 // ids (descending logit, lower id first among equal logits) and the softmax
 // probabilities over all 64 at those ids.
@@ -79,11 +68,7 @@ __device__ __forceinline__ void topk_softmax_warp(const float* l, int lane, int3
   }
 }
 
-// Decode sizes compute the logits inside the layer-entry kernel
-// (layer_entry.cuh): 16-expert slices of the router weights in shared memory as
-// padded quarter rows, four threads per (token, expert) output.
-constexpr int kRtExperts = 16;  // experts per router slice
-constexpr int kRtPad = 8;       // elements of padding per quarter row: conflict-free 16-byte reads
+// Decode sizes compute the logits inside the layer-entry kernel (layer_entry.cuh).
 
 // Large token counts: a 128-token x 64-expert block tile, staged through shared
 // memory 32 k at a time; each thread owns 8 tokens x 4 experts and runs every

@@ -138,7 +138,7 @@ bool dims_supported(const vg_moe_dims* d) {
 }
 
 struct MoeWs {
-  size_t idx, w, logits, offsets, perm, inv, xperm, act, o, ccnt, cbase, ecnt, sched, gbar, total;
+  size_t idx, w, offsets, perm, inv, xperm, act, o, ccnt, cbase, ecnt, sched, gbar, total;
   int sched_len;
 };
 
@@ -166,7 +166,6 @@ MoeWs moe_layout(int T) {
   };
   L.idx = take(N * 4);
   L.w = take(N * 4);
-  L.logits = take((size_t)T * kE * 4);
   L.offsets = take((kE + 1) * 4);
   L.perm = take(N * 4);
   L.inv = take(N * 4);
@@ -191,7 +190,7 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 // Device buffers of one layer inside the workspace (or the caller's taps).
 struct LayerBufs {
   int32_t *idx, *offsets, *perm, *inv, *sched, *ccnt, *cbase, *ecnt;
-  float *gw, *logits;
+  float* gw;
   uint32_t* gbar;
   __nv_bfloat16 *xperm, *act, *o;
   int sched_len;
@@ -209,7 +208,6 @@ LayerBufs carve(void* workspace, int T, const vg_moe_taps* taps) {
   b.act = (taps && taps->act) ? static_cast<__nv_bfloat16*>(taps->act) : reinterpret_cast<__nv_bfloat16*>(ws + L.act);
   b.o = (taps && taps->expert_out) ? static_cast<__nv_bfloat16*>(taps->expert_out)
                                    : reinterpret_cast<__nv_bfloat16*>(ws + L.o);
-  b.logits = reinterpret_cast<float*>(ws + L.logits);
   b.xperm = reinterpret_cast<__nv_bfloat16*>(ws + L.xperm);
   b.sched = reinterpret_cast<int32_t*>(ws + L.sched);
   b.sched_len = L.sched_len;
