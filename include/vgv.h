@@ -101,8 +101,10 @@ int32_t vg_abi_version(void);
 size_t vg_moe_workspace_bytes(const vg_moe_dims* dims, int32_t T_max);
 
 /* One MoE feed-forward layer over T tokens.
- *   logits l[t,e] = fp32 fma chain over h = 0..H-1 of x[t,h]*router_w[e,h]
- *                   starting at +0, then + router_bias[e] (fp32) if given;
+ *   logits l[t,e] = (q0 + q1) + (q2 + q3) in fp32, q_i = fp32 fma chain of
+ *                   x[t,h]*router_w[e,h] over the i-th contiguous quarter of h
+ *                   in increasing h, starting at +0; then + router_bias[e]
+ *                   (fp32) if given;
  *   idx   = the top_k experts by (l descending, e ascending);
  *   g     = softmax over all E logits at idx (no renormalisation);
  *   y[t]  = sum_j g[t,j] * SwiGLU_{idx[t,j]}(x[t]) + sum_s SwiGLU^shared_s(x[t]),
