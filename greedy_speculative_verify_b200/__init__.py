@@ -28,7 +28,8 @@ EXPORTS = (
     "vg_moe_stack_workspace_bytes", "vg_moe_ffn_stack", "vg_verify_workspace_bytes",
     "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag",
     "vg_profile_set_events", "vg_profile_count", "vg_verify_greedy_noalloc",
-    "vg_embed_rows", "vg_spec_rows", "vg_spec_commit",
+    "vg_embed_rows", "vg_spec_rows", "vg_spec_commit", "vg_spec_rows_given",
+    "vg_mtp_workspace_bytes", "vg_mtp_draft",
 )
 
 # vg_kernel
@@ -59,6 +60,12 @@ class vg_spec_state(ctypes.Structure):
                 ("cap", ctypes.c_int32), ("ref", ctypes.c_void_p), ("ref_len", ctypes.c_int32),
                 ("p", ctypes.c_float), ("seed", ctypes.c_uint64), ("step", ctypes.c_void_p),
                 ("tokens", ctypes.c_void_p), ("drafts", ctypes.c_void_p)]
+
+
+class vg_mtp_weights(ctypes.Structure):
+    _fields_ = [("proj", ctypes.c_void_p), ("ffn", ctypes.c_void_p), ("gamma_h", ctypes.c_void_p),
+                ("gamma_e", ctypes.c_void_p), ("gamma_f", ctypes.c_void_p), ("emb", ctypes.c_void_p),
+                ("lm_head", ctypes.c_void_p), ("V", ctypes.c_int32)]
 
 
 MOE_DIMS = vg_moe_dims(1280, 896, 64, 2, 6)
@@ -95,6 +102,9 @@ def load():
         "vg_embed_rows": (i32, [vp, i32, vp, i32, i32, vp, vp]),
         "vg_spec_rows": (i32, [ctypes.POINTER(vg_spec_state), vp]),
         "vg_spec_commit": (i32, [ctypes.POINTER(vg_spec_state), vp, vp, vp]),
+        "vg_spec_rows_given": (i32, [ctypes.POINTER(vg_spec_state), vp]),
+        "vg_mtp_workspace_bytes": (sz, [i32, i32]),
+        "vg_mtp_draft": (i32, [i32, i32, ctypes.POINTER(vg_mtp_weights), vp, i32, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -245,3 +255,27 @@ def vg_spec_rows(state, stream=None):
 def vg_spec_commit(state, accepted, out_tokens, stream=None):
     _check(load().vg_spec_commit(ctypes.byref(state), _ptr(accepted), _ptr(out_tokens), _stream(stream)),
            "vg_spec_commit")
+
+
+def vg_spec_rows_given(state, stream=None):
+    _check(load().vg_spec_rows_given(ctypes.byref(state), _stream(stream)), "vg_spec_rows_given")
+
+
+# ------------------------------------------------------------ draft block
+def make_mtp_weights(proj, ffn, gamma_h, gamma_e, gamma_f, emb, lm_head):
+    """vg_mtp_weights over caller-owned device tensors (fp32 gammas, bf16 rest)."""
+    for t in (proj, ffn, gamma_h, gamma_e, gamma_f, emb, lm_head):
+        if not t.is_contiguous():
+            raise ValueError("vg_mtp_weights tensors must be contiguous")
+    return vg_mtp_weights(proj.data_ptr(), ffn.data_ptr(), gamma_h.data_ptr(), gamma_e.data_ptr(),
+                          gamma_f.data_ptr(), emb.data_ptr(), lm_head.data_ptr(), lm_head.shape[0])
+
+
+def vg_mtp_workspace_bytes(B, V):
+    return load().vg_mtp_workspace_bytes(B, V)
+
+
+def vg_mtp_draft(B, K, weights, h, rows_per_seq, accepted, y0, drafts, workspace, hidden_out=None, stream=None):
+    _check(load().vg_mtp_draft(B, K, ctypes.byref(weights), _ptr(h), rows_per_seq, _ptr(accepted), _ptr(y0),
+                               _ptr(drafts), _ptr(hidden_out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "vg_mtp_draft")

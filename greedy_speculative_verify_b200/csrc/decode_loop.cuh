@@ -85,6 +85,17 @@ __global__ void __launch_bounds__(128) spec_rows(const SpecState s) {
   }
 }
 
+// Rows from drafts already in s.drafts (written by another drafter).
+__global__ void __launch_bounds__(128) spec_rows_given(const SpecState s) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= s.B) return;
+  const int K1 = s.K + 1;
+  s.tokens[(size_t)b * K1] = s.last[b];
+  for (int i = 1; i <= s.K; ++i) s.tokens[(size_t)b * K1 + i] = s.drafts[(size_t)b * s.K + i - 1];
+}
+
 __global__ void __launch_bounds__(128) spec_commit(const SpecState s, const int32_t* __restrict__ accepted,
                                                    const int32_t* __restrict__ out_tokens) {
   griddep_launch_dependents();

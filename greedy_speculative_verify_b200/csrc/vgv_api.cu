@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "combine.cuh"
 #include "decode_loop.cuh"
+#include "mtp.cuh"
 #include "gemm_moe.cuh"
 #include "layer_entry.cuh"
 #include "lmhead.cuh"
@@ -765,4 +766,166 @@ extern "C" vg_status vg_spec_commit(const vg_spec_state* st, const int32_t* acce
   const cudaError_t e = launch_dep(vg::spec_commit, vg::cdiv(st->B, 128), 128, 0,
                                    reinterpret_cast<cudaStream_t>(stream), Launch::kPlain, spec_dev(st), accepted, out_tokens);
   return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+extern "C" vg_status vg_spec_rows_given(const vg_spec_state* st, vg_stream_t stream) {
+  if (!spec_state_ok(st)) return VG_ERR_INVALID_ARG;
+  if (st->B == 0) return VG_OK;
+  const cudaError_t e = launch_dep(vg::spec_rows_given, vg::cdiv(st->B, 128), 128, 0,
+                                   reinterpret_cast<cudaStream_t>(stream), Launch::kPlain, spec_dev(st));
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ draft block
+namespace {
+// One dense product y = W x on the expert GEMM kernel, as a single shared
+// expert over T token rows (no routed experts, offsets[0] = 0):
+//  * with_gu: w is an expert block (gate | up | down), x the [T, H] input rows,
+//    act a [T, I] scratch for the SwiGLU activations: out = FFN(x);
+//  * otherwise w is [H, k_dn] and acts as the down projection of a unit list
+//    with no gate/up units (no readiness to wait for): out = w act, act the
+//    [T, k_dn] input rows.
+vg_status launch_dense(DevState* dev, int T, const void* w, bool with_gu, int k_dn, const void* x, void* act,
+                       void* out, int32_t* sched, int32_t* zero_offsets, cudaStream_t s) {
+  using namespace vg;
+  const int nt = expert_tile(T), bx = std::min(kBoxRows, nt);
+  const int tiles = cdiv(T, nt);
+  const uint64_t block = with_gu ? (uint64_t)3 * kI * kH * 2 : (uint64_t)kH * k_dn * 2;
+  const uint8_t* w8 = static_cast<const uint8_t*>(w);
+  const void* wdn = with_gu ? static_cast<const void*>(w8 + (size_t)2 * kI * kH * 2) : w;
+  CUtensorMap mGu, mDn, mX, mAct;
+  const uint64_t dGu[4] = {kH, kI, 2, 1}, sGu[3] = {kH * 2, (uint64_t)kI * kH * 2, (uint64_t)3 * kI * kH * 2};
+  const uint32_t bGu[4] = {kBK, kBM, 2, 1};
+  const uint64_t dDn[3] = {(uint64_t)k_dn, kH, 1}, sDn[2] = {(uint64_t)k_dn * 2, block};
+  const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
+  const void* xs = with_gu ? x : act;  // without gate/up the x map is never read
+  const uint64_t dX[2] = {kH, (uint64_t)T}, sX[1] = {(uint64_t)(with_gu ? kH : k_dn) * 2};
+  const uint32_t bX[2] = {kBK, (uint32_t)box_rows(T, bx)};
+  const uint64_t dAct[2] = {(uint64_t)k_dn, (uint64_t)T}, sAct[1] = {(uint64_t)k_dn * 2};
+  const uint32_t bAct[2] = {kBK, (uint32_t)box_rows(T, bx)};
+  // without gate/up the gate/up map is never read either: any valid map will do
+  if (make_map(&mGu, with_gu ? w : wdn, 4, dGu, sGu, bGu) || make_map(&mDn, wdn, 3, dDn, sDn, bDn) ||
+      make_map(&mX, xs, 2, dX, sX, bX) || make_map(&mAct, act, 2, dAct, sAct, bAct))
+    return VG_ERR_CUDA;
+  FusedArgs a{};
+  a.offsets = zero_offsets;
+  a.T = T;
+  a.E = 0;
+  a.S = 1;
+  a.mblk_gu = with_gu ? kI / kBM : 0;
+  a.mblk_dn = kH / (2 * kBM);
+  a.kc_gu = kH / kBK;
+  a.kc_dn = k_dn / kBK;
+  a.box_xr = (int)bX[1];
+  a.box_xs = (int)bX[1];
+  a.box_act = (int)bAct[1];
+  a.sched = sched;
+  a.act = static_cast<__nv_bfloat16*>(act);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  if (cudaMemsetAsync(sched, 0, (size_t)(1 + tiles) * 4, s) != cudaSuccess) return cuda_fail();
+  const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * tiles);
+  auto go = [&](auto kern, int smem) {
+    return launch_dep(kern, grid, 192, smem, s, Launch::kPlain, mGu, mGu, mDn, mDn, mX, mX, mAct, a);
+  };
+  const cudaError_t e = nt == 16   ? go(moe_expert_gemms<16>, FgCfg<16>::kSmemBytes)
+                        : nt == 64 ? go(moe_expert_gemms<64>, FgCfg<64>::kSmemBytes)
+                                   : go(moe_expert_gemms<128>, FgCfg<128>::kSmemBytes);
+  return e == cudaSuccess ? VG_OK : VG_ERR_CUDA;
+}
+
+struct MtpWs {
+  size_t u, z, zn, act, o, g, sched, zero, arg, acc, tok, vws, total;
+};
+MtpWs mtp_layout(int B, int V) {
+  MtpWs L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.u = take((size_t)B * 2 * kH * 2);
+  L.z = take((size_t)B * kH * 2);
+  L.zn = take((size_t)B * kH * 2);
+  L.act = take((size_t)B * kI * 2);
+  L.o = take((size_t)B * kH * 2);
+  L.g = take((size_t)B * kH * 2);
+  L.sched = take((size_t)(2 + vg::cdiv(B, 16)) * 4);
+  L.zero = take(16);
+  L.arg = take((size_t)B * 4);
+  L.acc = take((size_t)B * 4);
+  L.tok = take((size_t)B * 4);
+  L.vws = take(verify_ws_bytes(B, 0, V));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+extern "C" size_t vg_mtp_workspace_bytes(int32_t B, int32_t V) {
+  if (B < 0 || V < 1) return 0;
+  return mtp_layout(B, V).total;
+}
+
+extern "C" vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void* h, int32_t rows_per_seq,
+                                  const int32_t* accepted, const int32_t* y0, int32_t* drafts, void* hidden_out,
+                                  void* workspace, size_t workspace_bytes, vg_stream_t stream) {
+  using namespace vg;
+  if (B < 0 || K < 0 || w == nullptr || w->V < 1 || rows_per_seq < 1) return VG_ERR_INVALID_ARG;
+  if (B == 0 || K == 0) return VG_OK;
+  if (!w->proj || !w->ffn || !w->gamma_h || !w->gamma_e || !w->gamma_f || !w->emb || !w->lm_head || !h || !y0 ||
+      !drafts)
+    return VG_ERR_INVALID_ARG;
+  if (!aligned16(w->proj) || !aligned16(w->ffn) || !aligned16(w->emb) || !aligned16(w->lm_head) || !aligned16(h) ||
+      !aligned16(hidden_out))
+    return VG_ERR_INVALID_ARG;
+  const MtpWs L = mtp_layout(B, w->V);
+  if (workspace == nullptr || workspace_bytes < L.total) return VG_ERR_WORKSPACE;
+  DevState* dev = nullptr;
+  vg_status st = device_state(&dev);
+  if (st != VG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(ws + o); };
+  auto i32 = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
+  if (cudaMemsetAsync(ws + L.zero, 0, 16, s) != cudaSuccess) return cuda_fail();
+  // g_i: in the caller's hidden_out when given, else in the workspace
+  auto g_of = [&](int i) {
+    return hidden_out ? static_cast<__nv_bfloat16*>(hidden_out) + (size_t)(i - 1) * B * kH : bf(L.g);
+  };
+  for (int i = 1; i <= K; ++i) {
+    MtpPrep p{};
+    p.g = i == 1 ? static_cast<const __nv_bfloat16*>(h) : g_of(i - 1);
+    p.rows_per_seq = i == 1 ? rows_per_seq : 1;
+    p.acc = i == 1 ? accepted : nullptr;
+    p.y = i == 1 ? y0 : i32(L.arg);
+    p.emb = static_cast<const __nv_bfloat16*>(w->emb);
+    p.V = w->V;
+    p.H = kH;
+    p.gamma_h = w->gamma_h;
+    p.gamma_e = w->gamma_e;
+    p.u = bf(L.u);
+    p.drafts = i == 1 ? nullptr : drafts;
+    p.K = K;
+    p.slot = i - 2;
+    if (launch_dep(mtp_prep, B, kMtpThreads, 0, s, Launch::kPlain, p) != cudaSuccess) return cuda_fail();
+    if ((st = launch_dense(dev, B, w->proj, false, 2 * kH, nullptr, bf(L.u), bf(L.z), i32(L.sched), i32(L.zero),
+                           s)) != VG_OK)
+      return st;
+    if (launch_dep(mtp_rmsnorm, B, kMtpThreads, 0, s, Launch::kPlain, (const __nv_bfloat16*)bf(L.z), w->gamma_f,
+                   (int)kH, bf(L.zn)) != cudaSuccess)
+      return cuda_fail();
+    if ((st = launch_dense(dev, B, w->ffn, true, kI, bf(L.zn), bf(L.act), bf(L.o), i32(L.sched), i32(L.zero), s)) !=
+        VG_OK)
+      return st;
+    if (launch_dep(mtp_residual, cdiv(B * kH / 8, 256), 256, 0, s, Launch::kPlain, (const __nv_bfloat16*)bf(L.z),
+                   (const __nv_bfloat16*)bf(L.o), B * kH, g_of(i)) != cudaSuccess)
+      return cuda_fail();
+    if ((st = vg_verify_greedy(B, 0, kH, w->V, g_of(i), w->lm_head, nullptr, i32(L.arg), i32(L.acc), i32(L.tok),
+                               ws + L.vws, verify_ws_bytes(B, 0, w->V), stream)) != VG_OK)
+      return st;
+  }
+  if (launch_dep(mtp_collect, cdiv(B, 128), 128, 0, s, Launch::kPlain, (const int32_t*)i32(L.arg), (int)B, (int)K,
+                 (int)K - 1, drafts) != cudaSuccess)
+    return cuda_fail();
+  return VG_OK;
 }

@@ -297,6 +297,54 @@ vg_status vg_spec_rows(const vg_spec_state* st, vg_stream_t stream);
 vg_status vg_spec_commit(const vg_spec_state* st, const int32_t* accepted, const int32_t* out_tokens,
                          vg_stream_t stream);
 
+/* Next verify rows from drafts the caller (e.g. vg_mtp_draft) has written to
+ * st->drafts: tokens[b] = [last[b], drafts[b, 0..K-1]]; st->ref and st->p are
+ * not used. Errors: VG_ERR_INVALID_ARG, VG_ERR_CUDA. */
+vg_status vg_spec_rows_given(const vg_spec_state* st, vg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Recursive draft block (FastMTP): one dense block reused for every draft
+ * step, fed back its own hidden state and its own last token ("Jina AI's 3.4B
+ * OCR model targets faster page parsing", "FastMTP cuts decoding work";
+ * "jina-ocr-v1: Schnellere Dokumentenanalyse auf kostengünstigen GPUs",
+ * "Modell und Training", "Erste Schritte"). The pages do not describe the
+ * block; the reading computed, step i = 1..K from (g, y) = (g_{i-1}, y_{i-1}):
+ *   u   = [rmsnorm(g) * gamma_h ; rmsnorm(emb[y]) * gamma_e]   bf16 [2H]
+ *   z   = proj u                                              bf16 [H]
+ *   g_i = bf16(z + FFN(rmsnorm(z) * gamma_f))                 bf16 [H]
+ *   y_i = argmax over v of lm_head[v] . g_i (fp32 decision, lowest index on ties)
+ * rmsnorm(x) = x / sqrt(mean(x^2) + 1e-6) in fp32; FFN = SwiGLU with one expert's
+ * layout and width (gate [I,H] | up [I,H] | down [H,I], I = 896), its
+ * activations rounded to bf16. g_0 is the given hidden row of each sequence
+ * (for a verify step: the row whose argmax was the bonus token), y_0 the given
+ * token (the bonus token). H = 1280.
+ * ------------------------------------------------------------------------- */
+typedef struct vg_mtp_weights {
+  const void* proj;       /* bf16 [H, 2H] */
+  const void* ffn;        /* bf16 [3 * I * H]: gate | up | down */
+  const float* gamma_h;   /* fp32 [H] */
+  const float* gamma_e;   /* fp32 [H] */
+  const float* gamma_f;   /* fp32 [H] */
+  const void* emb;        /* bf16 [V, H] token embedding */
+  const void* lm_head;    /* bf16 [V, H] (the verifier's) */
+  int32_t V;
+} vg_mtp_weights;
+
+/* Workspace of vg_mtp_draft for up to B sequences; 0 if B < 0 or V < 1. */
+size_t vg_mtp_workspace_bytes(int32_t B, int32_t V);
+
+/* K draft steps for B sequences. h: bf16 rows; the row of sequence b is
+ * b * rows_per_seq + (accepted ? accepted[b] : 0) (pass a verify step's hidden
+ * states, K+1 and its accepted lengths). y0 int32 [B]. drafts int32 [B, K]
+ * receives y_1 .. y_K; hidden_out, if not NULL, bf16 [K, B, H] receives
+ * g_1 .. g_K. K = 0 or B = 0 is a no-op. Stream-ordered, capturable.
+ * Errors: VG_ERR_INVALID_ARG, VG_ERR_WORKSPACE, VG_ERR_CUDA; a token outside
+ * [0, V) or an accepted length outside [0, rows_per_seq) records
+ * VG_ERR_DEVICE_BOUNDS. */
+vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void* h, int32_t rows_per_seq,
+                       const int32_t* accepted, const int32_t* y0, int32_t* drafts, void* hidden_out,
+                       void* workspace, size_t workspace_bytes, vg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

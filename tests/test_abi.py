@@ -138,3 +138,21 @@ def test_decode_loop_validation_before_launch(lib):
     assert f_rows(ctypes.byref(mk(B=0)), None) == 0                                # B = 0: no-op
     assert f_commit(ctypes.byref(mk()), None, A, None) == 1                        # accepted needed
     assert f_commit(ctypes.byref(mk(B=0)), None, None, None) == 0
+
+
+def test_draft_block_validation_before_launch(lib):
+    A = 1 << 40
+    w = vgv.vg_mtp_weights(A, A, A, A, A, A, A, 1000)
+    need = vgv.vg_mtp_workspace_bytes(4, 1000)
+    assert need > 0 and vgv.vg_mtp_workspace_bytes(-1, 1000) == 0 and vgv.vg_mtp_workspace_bytes(4, 0) == 0
+    f = lib.vg_mtp_draft
+    assert f(4, 0, ctypes.byref(w), A, 4, None, A, A, None, A, need, None) == 0       # K = 0: no-op
+    assert f(0, 3, ctypes.byref(w), A, 4, None, A, A, None, A, need, None) == 0       # B = 0: no-op
+    assert f(-1, 3, ctypes.byref(w), A, 4, None, A, A, None, A, need, None) == 1
+    assert f(4, 3, None, A, 4, None, A, A, None, A, need, None) == 1
+    assert f(4, 3, ctypes.byref(w), A, 0, None, A, A, None, A, need, None) == 1       # rows_per_seq >= 1
+    assert f(4, 3, ctypes.byref(w), None, 4, None, A, A, None, A, need, None) == 1    # h needed
+    assert f(4, 3, ctypes.byref(w), A + 8, 4, None, A, A, None, A, need, None) == 1   # misaligned h
+    assert f(4, 3, ctypes.byref(w), A, 4, None, A, A, None, A, need - 1, None) == 3   # short workspace
+    bad = vgv.vg_mtp_weights(A, None, A, A, A, A, A, 1000)
+    assert f(4, 3, ctypes.byref(bad), A, 4, None, A, A, None, A, need, None) == 1     # ffn needed

@@ -30,9 +30,11 @@ class Decoder:
         self.emb = si.torch_normal_bf16((V, D.H), 1.0, 0, cfg, si.TID_EMB)
         self.lm = si.torch_normal_bf16((V, D.H), 0.02, 0, cfg, si.TID_LM_HEAD)
 
-    def run(self, starts, K, n_tokens, ref=None, p=0.0, seed=1, graph=False):
+    def run(self, starts, K, n_tokens, ref=None, p=0.0, seed=1, graph=False, mtp=None):
         """Decodes until every sequence has n_tokens committed; returns
-        (committed [B, n_tokens], accepted lengths per step [steps, B])."""
+        (committed [B, n_tokens], accepted lengths per step [steps, B]). With
+        mtp (draft-block weights), the drafts of every step after the first come
+        from the draft block fed the previous verify step's hidden states."""
         B = starts.numel()
         T = B * (K + 1)
         i32 = dict(dtype=torch.int32, device="cuda")
@@ -50,12 +52,21 @@ class Decoder:
         ew = [l["expert_w"] for l in self.layers]
         sw = [l["shared_w"] for l in self.layers]
 
+        ws_m = torch.empty(vgv.vg_mtp_workspace_bytes(B, V), dtype=torch.uint8, device="cuda") if mtp else None
+        first = [True]
+
         def one_step():
-            vgv.vg_spec_rows(st)
+            if mtp is None or first[0]:
+                vgv.vg_spec_rows(st)
+            else:
+                vgv.vg_spec_rows_given(st)
+            first[0] = False
             vgv.vg_embed_rows(tokens.view(-1), self.emb, x)
             vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, len(self.layers), T, x, rw, None, ew, sw, hid, ws_s)
             vgv.vg_verify_greedy(B, K, D.H, V, hid, self.lm, drafts if K else None, argmax, accepted, out, ws_v)
             vgv.vg_spec_commit(st, accepted, out)
+            if mtp is not None:
+                vgv.vg_mtp_draft(B, K, mtp, hid, K + 1, accepted, last, drafts, ws_m)
 
         g = None
         if graph:
