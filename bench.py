@@ -157,7 +157,15 @@ def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
     starts = torch.randint(0, V, (B,), generator=g, device=dev, dtype=torch.int32)
     stream = torch.cuda.current_stream()
 
-    def loop(K, n_tokens, ref=None, steps=None):
+    # draft-block weights (synthetic: the drafts are rarely accepted, the cost is real)
+    mtp_t = {
+        "proj": si.torch_normal_bf16((H, 2 * H), 0.02, SEED, CFG, si.TID_EMB, 1, device=dev),
+        "ffn": si.torch_normal_bf16((3 * I * H,), 0.02, SEED, CFG, si.TID_EMB, 2, device=dev),
+        "g": [torch.ones(H, dtype=torch.float32, device=dev) for _ in range(3)],
+    }
+    mtp_w = vgv.make_mtp_weights(mtp_t["proj"], mtp_t["ffn"], *mtp_t["g"], emb, lm)
+
+    def loop(K, n_tokens, ref=None, steps=None, mtp=False):
         T_ = B * (K + 1)
         last, pos, step = starts.clone(), torch.zeros(B, **i32), torch.zeros(1, **i32)
         cap = n_tokens + (K + 1) * ((steps or 0) + 5) + K + 1  # every step of the run fits
@@ -170,14 +178,23 @@ def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
         ws_v = torch.empty(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
         st = vgv.make_spec_state(B, K, V, last, pos, committed, ref, p, SEED + 29, step, tokens, drafts if K else None)
 
-        def one():
-            vgv.vg_spec_rows(st)
+        ws_m = torch.empty(vgv.vg_mtp_workspace_bytes(B, V), dtype=torch.uint8, device=dev) if mtp else None
+
+        def one(rows=True):
+            if rows:
+                vgv.vg_spec_rows(st) if not mtp else vgv.vg_spec_rows_given(st)
             vgv.vg_embed_rows(tokens.view(-1), emb, x)
             vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, T_, x, rw, None, ew, sw, hid, ws_s)
             vgv.vg_verify_greedy(B, K, H, V, hid, lm, drafts if K else None, am, acc, out, ws_v)
             vgv.vg_spec_commit(st, acc, out)
+            if mtp:  # the next step's drafts from the draft block at this step's hidden states
+                vgv.vg_mtp_draft(B, K, mtp_w, hid, K + 1, acc, last, drafts, ws_m)
 
-        one()
+        if mtp:  # first rows: uniform drafts
+            vgv.vg_spec_rows(st)
+            one(rows=False)
+        else:
+            one()
         torch.cuda.synchronize()
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr):
@@ -205,11 +222,18 @@ def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
     spec, tokens_timed, ms = loop(K, 0, ref=greedy, steps=n_steps)
     n_cmp = min(int((spec >= 0).sum(1).min()), ref_len)
     lossless = bool(torch.equal(spec[:, :n_cmp], greedy[:, :n_cmp]))
+    spec_m, tok_m, ms_m = loop(K, 0, steps=n_steps, mtp=True)
+    n_cmp_m = min(int((spec_m >= 0).sum(1).min()), ref_len)
+    lossless_m = bool(torch.equal(spec_m[:, :n_cmp_m], greedy[:, :n_cmp_m]))
     return {"workload": f"B={B} sequences, K={K}, {LAYERS} layers, V={V}: device loop of draft rows, embedding, "
                         f"MoE stack, verify, commit (CUDA graph), {n_steps} timed steps",
             "tokens_per_s": tokens_timed / (ms * n_steps / 1e3), "ms_per_step": ms,
             "tau": tokens_timed / (B * n_steps), "draft_p": p,
-            "lossless_vs_greedy": lossless, "tokens_compared": n_cmp * B}
+            "lossless_vs_greedy": lossless, "tokens_compared": n_cmp * B,
+            "draft_block": {"ms_per_step": ms_m, "tau": tok_m / (B * n_steps),
+                            "lossless_vs_greedy": lossless_m, "tokens_compared": n_cmp_m * B,
+                            "note": "drafts from the recursive draft block (synthetic weights) at each verify "
+                                    "step's hidden states; ms_per_step includes its K draft steps"}}
 
 
 def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
