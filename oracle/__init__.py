@@ -46,10 +46,12 @@ from .experts import silu, swiglu_expert, moe_ffn, moe_stack
 from .verify import lm_head_argmax, logit_fp64, prefix_accept, tau, acceptance_rate
 from .decode import MarkovDecoder, greedy_decode, speculative_decode
 from .mtp import rmsnorm, mtp_step, mtp_draft
+from .attention import rope, attn_verify
 
 __all__ = [
     "widen", "round_bf16_bits", "router_logits", "route", "softmax_gates", "segment_bounds",
     "expert_permutation", "silu", "swiglu_expert", "moe_ffn", "moe_stack",
     "lm_head_argmax", "logit_fp64", "prefix_accept", "tau", "acceptance_rate",
     "MarkovDecoder", "greedy_decode", "speculative_decode", "rmsnorm", "mtp_step", "mtp_draft",
+    "rope", "attn_verify",
 ]
