@@ -29,7 +29,7 @@ EXPORTS = (
     "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag",
     "vg_profile_set_events", "vg_profile_count", "vg_verify_greedy_noalloc",
     "vg_embed_rows", "vg_spec_rows", "vg_spec_commit", "vg_spec_rows_given",
-    "vg_mtp_workspace_bytes", "vg_mtp_draft",
+    "vg_mtp_workspace_bytes", "vg_mtp_draft", "vg_attn_workspace_bytes", "vg_attn_verify",
 )
 
 # vg_kernel
@@ -105,6 +105,8 @@ def load():
         "vg_spec_rows_given": (i32, [ctypes.POINTER(vg_spec_state), vp]),
         "vg_mtp_workspace_bytes": (sz, [i32, i32]),
         "vg_mtp_draft": (i32, [i32, i32, ctypes.POINTER(vg_mtp_weights), vp, i32, vp, vp, vp, vp, vp, sz, vp]),
+        "vg_attn_workspace_bytes": (sz, [i32, i32, i32]),
+        "vg_attn_verify": (i32, [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -279,3 +281,15 @@ def vg_mtp_draft(B, K, weights, h, rows_per_seq, accepted, y0, drafts, workspace
     _check(load().vg_mtp_draft(B, K, ctypes.byref(weights), _ptr(h), rows_per_seq, _ptr(accepted), _ptr(y0),
                                _ptr(drafts), _ptr(hidden_out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "vg_mtp_draft")
+
+
+# ------------------------------------------------------------ verifier attention
+def vg_attn_workspace_bytes(B, K, L_max):
+    return load().vg_attn_workspace_bytes(B, K, L_max)
+
+
+def vg_attn_verify(B, K, x, w_qkv, w_o, kv_cache, lens, out, workspace, o_out=None, stream=None):
+    """One attention layer of a verify step; kv_cache [B, 2, L_max, H]."""
+    _check(load().vg_attn_verify(B, K, kv_cache.shape[2], _ptr(x), _ptr(w_qkv), _ptr(w_o), _ptr(kv_cache), _ptr(lens),
+                                 _ptr(out), _ptr(o_out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "vg_attn_verify")

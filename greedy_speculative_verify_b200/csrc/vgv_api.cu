@@ -13,6 +13,7 @@
 #include "combine.cuh"
 #include "decode_loop.cuh"
 #include "mtp.cuh"
+#include "attention.cuh"
 #include "gemm_moe.cuh"
 #include "layer_entry.cuh"
 #include "lmhead.cuh"
@@ -782,21 +783,21 @@ namespace {
 // expert over T token rows (no routed experts, offsets[0] = 0):
 //  * with_gu: w is an expert block (gate | up | down), x the [T, H] input rows,
 //    act a [T, I] scratch for the SwiGLU activations: out = FFN(x);
-//  * otherwise w is [H, k_dn] and acts as the down projection of a unit list
-//    with no gate/up units (no readiness to wait for): out = w act, act the
-//    [T, k_dn] input rows.
-vg_status launch_dense(DevState* dev, int T, const void* w, bool with_gu, int k_dn, const void* x, void* act,
-                       void* out, int32_t* sched, int32_t* zero_offsets, cudaStream_t s) {
+//  * otherwise w is [n_out, k_dn] (n_out a multiple of 256) and acts as the
+//    down projection of a unit list with no gate/up units (no readiness to wait
+//    for): out [T, n_out] = act w^T, act the [T, k_dn] input rows.
+vg_status launch_dense(DevState* dev, int T, const void* w, bool with_gu, int k_dn, int n_out, const void* x,
+                       void* act, void* out, int32_t* sched, int32_t* zero_offsets, cudaStream_t s) {
   using namespace vg;
   const int nt = expert_tile(T), bx = std::min(kBoxRows, nt);
   const int tiles = cdiv(T, nt);
-  const uint64_t block = with_gu ? (uint64_t)3 * kI * kH * 2 : (uint64_t)kH * k_dn * 2;
+  const uint64_t block = with_gu ? (uint64_t)3 * kI * kH * 2 : (uint64_t)n_out * k_dn * 2;
   const uint8_t* w8 = static_cast<const uint8_t*>(w);
   const void* wdn = with_gu ? static_cast<const void*>(w8 + (size_t)2 * kI * kH * 2) : w;
   CUtensorMap mGu, mDn, mX, mAct;
   const uint64_t dGu[4] = {kH, kI, 2, 1}, sGu[3] = {kH * 2, (uint64_t)kI * kH * 2, (uint64_t)3 * kI * kH * 2};
   const uint32_t bGu[4] = {kBK, kBM, 2, 1};
-  const uint64_t dDn[3] = {(uint64_t)k_dn, kH, 1}, sDn[2] = {(uint64_t)k_dn * 2, block};
+  const uint64_t dDn[3] = {(uint64_t)k_dn, (uint64_t)n_out, 1}, sDn[2] = {(uint64_t)k_dn * 2, block};
   const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
   const void* xs = with_gu ? x : act;  // without gate/up the x map is never read
   const uint64_t dX[2] = {kH, (uint64_t)T}, sX[1] = {(uint64_t)(with_gu ? kH : k_dn) * 2};
@@ -813,7 +814,7 @@ vg_status launch_dense(DevState* dev, int T, const void* w, bool with_gu, int k_
   a.E = 0;
   a.S = 1;
   a.mblk_gu = with_gu ? kI / kBM : 0;
-  a.mblk_dn = kH / (2 * kBM);
+  a.mblk_dn = n_out / (2 * kBM);
   a.kc_gu = kH / kBK;
   a.kc_dn = k_dn / kBK;
   a.box_xr = (int)bX[1];
@@ -908,14 +909,14 @@ extern "C" vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w,
     p.K = K;
     p.slot = i - 2;
     if (launch_dep(mtp_prep, B, kMtpThreads, 0, s, Launch::kPlain, p) != cudaSuccess) return cuda_fail();
-    if ((st = launch_dense(dev, B, w->proj, false, 2 * kH, nullptr, bf(L.u), bf(L.z), i32(L.sched), i32(L.zero),
-                           s)) != VG_OK)
+    if ((st = launch_dense(dev, B, w->proj, false, 2 * kH, kH, nullptr, bf(L.u), bf(L.z), i32(L.sched),
+                           i32(L.zero), s)) != VG_OK)
       return st;
     if (launch_dep(mtp_rmsnorm, B, kMtpThreads, 0, s, Launch::kPlain, (const __nv_bfloat16*)bf(L.z), w->gamma_f,
                    (int)kH, bf(L.zn)) != cudaSuccess)
       return cuda_fail();
-    if ((st = launch_dense(dev, B, w->ffn, true, kI, bf(L.zn), bf(L.act), bf(L.o), i32(L.sched), i32(L.zero), s)) !=
-        VG_OK)
+    if ((st = launch_dense(dev, B, w->ffn, true, kI, kH, bf(L.zn), bf(L.act), bf(L.o), i32(L.sched), i32(L.zero),
+                           s)) != VG_OK)
       return st;
     if (launch_dep(mtp_residual, cdiv(B * kH / 8, 256), 256, 0, s, Launch::kPlain, (const __nv_bfloat16*)bf(L.z),
                    (const __nv_bfloat16*)bf(L.o), B * kH, g_of(i)) != cudaSuccess)
@@ -926,6 +927,98 @@ extern "C" vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w,
   }
   if (launch_dep(mtp_collect, cdiv(B, 128), 128, 0, s, Launch::kPlain, (const int32_t*)i32(L.arg), (int)B, (int)K,
                  (int)K - 1, drafts) != cudaSuccess)
+    return cuda_fail();
+  return VG_OK;
+}
+
+// ------------------------------------------------------------ verifier attention
+namespace {
+struct AttnWs {
+  size_t qkv, q, o, proj, part, sched, zero, total;
+};
+AttnWs attn_layout(int B, int K, int L_max) {
+  const size_t R = (size_t)B * (K + 1);
+  AttnWs L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.qkv = take(R * 3 * kH * 2);
+  L.q = take(R * kH * 2);
+  L.o = take(R * kH * 2);
+  L.proj = take(R * kH * 2);
+  L.part = take((size_t)B * vg::kAttnHeads * vg::cdiv(L_max, vg::kAttnChunk) * (K + 1) * (2 + vg::kAttnDim) * 4);
+  L.sched = take((size_t)(2 + vg::cdiv((int)R, 16)) * 4);
+  L.zero = take(16);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+extern "C" size_t vg_attn_workspace_bytes(int32_t B, int32_t K, int32_t L_max) {
+  if (B < 0 || K < 0 || K + 1 > vg::kAttnMaxRows || L_max < 1 || L_max > 32768) return 0;
+  return attn_layout(B, K, L_max).total;
+}
+
+extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const void* x, const void* w_qkv,
+                                    const void* w_o, void* kv_cache, const int32_t* lens, void* out, void* o_out,
+                                    void* workspace, size_t workspace_bytes, vg_stream_t stream) {
+  using namespace vg;
+  if (B < 0 || K < 0 || K + 1 > kAttnMaxRows || L_max < 1 || L_max > 32768) return VG_ERR_INVALID_ARG;
+  if (B == 0) return VG_OK;
+  if (!x || !w_qkv || !w_o || !kv_cache || !lens || !out) return VG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(w_o) || !aligned16(kv_cache) || !aligned16(out) ||
+      !aligned16(o_out))
+    return VG_ERR_INVALID_ARG;
+  const int R = B * (K + 1);
+  if (overlaps(x, (size_t)R * kH * 2, out, (size_t)R * kH * 2)) return VG_ERR_INVALID_ARG;
+  const AttnWs L = attn_layout(B, K, L_max);
+  if (workspace == nullptr || workspace_bytes < L.total) return VG_ERR_WORKSPACE;
+  DevState* dev = nullptr;
+  vg_status st = device_state(&dev);
+  if (st != VG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(ws + o); };
+  auto i32 = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
+  if (cudaMemsetAsync(ws + L.zero, 0, 16, s) != cudaSuccess) return cuda_fail();
+  // qkv = x W_qkv^T: a down-only unit list with 3H output rows
+  if ((st = launch_dense(dev, R, w_qkv, false, kH, 3 * kH, nullptr, const_cast<void*>(x), bf(L.qkv), i32(L.sched),
+                         i32(L.zero), s)) != VG_OK)
+    return st;
+  AttnArgs a{};
+  a.B = B;
+  a.K1 = K + 1;
+  a.L_max = L_max;
+  a.lens = lens;
+  a.qkv = bf(L.qkv);
+  a.q = bf(L.q);
+  a.cache = static_cast<__nv_bfloat16*>(kv_cache);
+  a.part = reinterpret_cast<float*>(ws + L.part);
+  a.n_chunks = cdiv(L_max, kAttnChunk);
+  a.o = o_out ? static_cast<__nv_bfloat16*>(o_out) : bf(L.o);
+  if (launch_dep(attn_rope_append, cdiv(R * kH / 2, 256), 256, 0, s, Launch::kPlain, a) != cudaSuccess)
+    return cuda_fail();
+  cudaLaunchConfig_t cfg = {};  // 2-d grid: (sequence x head, chunk)
+  cfg.gridDim = dim3(B * kAttnHeads, a.n_chunks);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn_chunk, a) != cudaSuccess) return cuda_fail();
+  if (launch_dep(attn_merge, B * kAttnHeads * (K + 1), kAttnDim, 0, s, Launch::kPlain, a) != cudaSuccess)
+    return cuda_fail();
+  // out = x + W_o o
+  if ((st = launch_dense(dev, R, w_o, false, kH, kH, nullptr, a.o, bf(L.proj), i32(L.sched), i32(L.zero), s)) !=
+      VG_OK)
+    return st;
+  if (launch_dep(mtp_residual, cdiv(R * kH / 8, 256), 256, 0, s, Launch::kPlain, static_cast<const __nv_bfloat16*>(x),
+                 (const __nv_bfloat16*)bf(L.proj), R * kH, static_cast<__nv_bfloat16*>(out)) != cudaSuccess)
     return cuda_fail();
   return VG_OK;
 }

@@ -345,6 +345,32 @@ vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void
                        const int32_t* accepted, const int32_t* y0, int32_t* drafts, void* hidden_out,
                        void* workspace, size_t workspace_bytes, vg_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Verifier attention over a KV cache (one layer of a verify step). The pages
+ * give the decoder's 32,768-position limit (jina-ocr-v1 model card,
+ * architecture paragraph) but not its attention; the reading computed:
+ *   qkv = x W_qkv^T (W_qkv bf16 [3H, H]: q rows, k rows, v rows), bf16;
+ *   10 heads of 128; RoFormer rotary positions on q and k: pair (2j, 2j+1) of a
+ *   head at position p turned by p * 10000^(-2j/128); row i of sequence b sits
+ *   at position lens[b] + i;
+ *   the new rows' k (rotated) and v are written into the cache at positions
+ *   lens[b] .. lens[b] + K;
+ *   row i attends to positions 0 .. lens[b] + i, scores q.k / sqrt(128), softmax;
+ *   out = bf16(x + bf16(W_o o)) (W_o bf16 [H, H]).
+ * x, out bf16 [B*(K+1), H] (rows of sequence b at b*(K+1) ..); kv_cache bf16
+ * [B, 2, L_max, H] (k then v, a position's heads side by side); lens int32 [B]
+ * is read, not advanced (advance it by the committed tokens; a later step
+ * overwrites the positions of rejected drafts). K+1 <= 8, L_max <= 32768;
+ * lens[b] + K + 1 > L_max records VG_ERR_DEVICE_BOUNDS and gives o = 0 for that
+ * sequence. out must not overlap x. o_out, if not NULL, bf16 [B*(K+1), H]
+ * receives the heads' output o before the output projection. Errors: VG_ERR_INVALID_ARG,
+ * VG_ERR_WORKSPACE, VG_ERR_CUDA.
+ * ------------------------------------------------------------------------- */
+size_t vg_attn_workspace_bytes(int32_t B, int32_t K, int32_t L_max);
+vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const void* x, const void* w_qkv, const void* w_o,
+                         void* kv_cache, const int32_t* lens, void* out, void* o_out, void* workspace,
+                         size_t workspace_bytes, vg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -156,3 +156,20 @@ def test_draft_block_validation_before_launch(lib):
     assert f(4, 3, ctypes.byref(w), A, 4, None, A, A, None, A, need - 1, None) == 3   # short workspace
     bad = vgv.vg_mtp_weights(A, None, A, A, A, A, A, 1000)
     assert f(4, 3, ctypes.byref(bad), A, 4, None, A, A, None, A, need, None) == 1     # ffn needed
+
+
+def test_attention_validation_before_launch(lib):
+    A = 1 << 40
+    need = vgv.vg_attn_workspace_bytes(4, 3, 512)
+    assert need > 0 and vgv.vg_attn_workspace_bytes(4, 8, 512) == 0 and vgv.vg_attn_workspace_bytes(4, 3, 40000) == 0
+    f = lib.vg_attn_verify
+    args = lambda **kw: [kw.get(k, v) for k, v in dict(B=4, K=3, L=512, x=A, wq=A + (1 << 30), wo=A + (2 << 30),
+                                                          c=A + (3 << 30), lens=A + (4 << 30), out=A + (5 << 30),
+                                                          o=None, ws=A + (6 << 30), n=need, s=None).items()]
+    assert f(*args(B=0)) == 0
+    assert f(*args(K=8)) == 1                     # at most 8 new rows per sequence
+    assert f(*args(L=0)) == 1
+    assert f(*args(x=None)) == 1
+    assert f(*args(out=A + 64)) == 1              # out overlaps x
+    assert f(*args(wq=A + 8)) == 1                # misaligned weights
+    assert f(*args(n=need - 1)) == 3
