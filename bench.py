@@ -278,6 +278,70 @@ def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
     return res
 
 
+ATTN_CONTEXTS = (2048, 8192)  # cached positions per sequence
+
+
+def attention_bytes(L: int) -> int:
+    """Algorithmic bytes of one verifier attention layer at B = 32, K = 3 over
+    caches of L positions: the projections' weights (3H x H and H x H), the
+    keys and values of every visible position read once, the new rows' keys and
+    values written, the layer's input read and output written (bf16)."""
+    R = B * (K + 1)
+    return (4 * H * H + B * (L + K + 1) * 2 * H + B * (K + 1) * 2 * H + 2 * R * H) * 2
+
+
+def measure_attention(vgv, si, dev, reps=20, contexts=ATTN_CONTEXTS):
+    """One verifier attention layer (q/k/v projection, rotary append, chunked
+    attention, merge, output projection, residual) at B = 32, K = 3 over caches
+    of L positions, replayed from a CUDA graph and timed with CUDA events. Every
+    call rewrites the new rows' cache positions with the same values, so the
+    replays are identical; the caches exceed the 126 MB L2."""
+    import torch
+
+    res = {}
+    stream = torch.cuda.current_stream()
+    R = B * (K + 1)
+    x = si.torch_normal_bf16((R, H), 1.0, SEED, 5, si.TID_X, device=dev)
+    wqkv = si.torch_normal_bf16((3 * H, H), 0.02, SEED, 5, si.TID_ATTN_QKV, device=dev)
+    wo = si.torch_normal_bf16((H, H), 0.02, SEED, 5, si.TID_ATTN_O, device=dev)
+    out = torch.empty_like(x)
+    peak, _ = _peaks()
+    for L in contexts:
+        L_max = L + K + 1
+        cache = si.torch_normal_bf16((B, 2, L_max, H), 0.7, SEED, 5, si.TID_KV, layer=L, device=dev)
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        ws = torch.empty(vgv.vg_attn_workspace_bytes(B, K, L_max), dtype=torch.uint8, device=dev)
+
+        def layer():
+            vgv.vg_attn_verify(B, K, x, wqkv, wo, cache, lens, out, ws)
+
+        layer()
+        torch.cuda.synchronize()
+        st, info = vgv.vg_get_device_status()
+        if st != 0:
+            raise RuntimeError(f"attention layer: device status {st} {info}")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            layer()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        nbytes = attention_bytes(L)
+        res[f"L{L}"] = {"ms_per_layer": ms, "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                        "frac_of_measured_hbm": nbytes / (ms / 1e3) / 1e9 / peak}
+        del g, cache, ws
+    res["workload"] = ("one attention layer of a B=32, K=3 verify step: 128 rows, 10 heads x 128, rotary positions, "
+                       "causal over L cached + 4 new positions, CUDA graph")
+    return res
+
+
 def _cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -582,6 +646,7 @@ def run_gpu(args, rank, world, local):
     prefill = measure_prefill(vgv, si, dev) if not args.no_extra else None
     latency = measure_latency(vgv, x, rw, ew, sw, lm, dev) if not args.no_extra else None
     spec_loop = measure_spec_loop(vgv, si, rw, ew, sw, lm, dev) if not args.no_extra else None
+    attention = measure_attention(vgv, si, dev) if not args.no_extra else None
 
     # ---- aggregate over ranks (max time, summed tokens)
     ms, e2e_ms, tokens_all = aggregate_over_ranks(ms, e2e_ms, tokens_rank, world, dev)
@@ -612,6 +677,7 @@ def run_gpu(args, rank, world, local):
         "prefill": prefill,
         "batch1_latency": latency,
         "spec_decode_loop": spec_loop,
+        "attention_layer": attention,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -619,6 +685,21 @@ def run_gpu(args, rank, world, local):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_attention_only(L: int) -> int:
+    import torch
+
+    import greedy_speculative_verify_b200 as vgv
+    import synth_inputs as si
+    from greedy_speculative_verify_b200 import build as vbuild
+
+    if not vbuild.up_to_date():
+        vbuild.build()
+    vgv.load()
+    res = measure_attention(vgv, si, torch.device("cuda", 0), contexts=(L,))
+    print(json.dumps({"attention_layer": res}), flush=True)
     return 0
 
 
@@ -630,11 +711,15 @@ def main():
     ap.add_argument("--impl", choices=["vgv", "reference"], default="vgv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill and batch-1 measurements")
+    ap.add_argument("--attention-only", type=int, default=0, metavar="L",
+                    help="time only the attention layer over caches of L positions (one GPU) and print its figures")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = _env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.attention_only:
+        return run_attention_only(args.attention_only)
     return run_gpu(args, rank, world, local)
 
 

@@ -11,7 +11,8 @@
 // attn_rope_append: rotates q and k of the new rows, stores q, appends k and v.
 // attn_chunk: flash-decoding partials — one CTA per (sequence, head, chunk of
 //   kAttnChunk cache positions): the chunk's score max, exp-sum and
-//   exp-weighted value sum for each new row.
+//   exp-weighted value sum for each new row; every key and value of the chunk
+//   is read once for all K+1 rows.
 // attn_merge: merges a (sequence, head, row)'s chunk partials into o.
 // The projections run on the expert GEMM kernel (dense unit lists).
 #pragma once
@@ -74,113 +75,172 @@ __global__ void __launch_bounds__(256) attn_rope_append(const AttnArgs a) {
   vc[2 * pr + 1] = row[2 * H + 2 * pr + 1];
 }
 
-// grid (B * heads, n_chunks); each thread scores one cache position against
-// every new row, then each thread accumulates (row, dim) outputs.
-__global__ void __launch_bounds__(kAttnThreads) attn_chunk(const AttnArgs a) {
+__device__ __forceinline__ void attn_unpack8(const uint4 u, float (&f)[8]) {
+  f[0] = bf16_lo(u.x), f[1] = bf16_hi(u.x), f[2] = bf16_lo(u.y), f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z), f[5] = bf16_hi(u.z), f[6] = bf16_lo(u.w), f[7] = bf16_hi(u.w);
+}
+
+// Sum of v[0 .. N) over the 2^NS lanes lane ^ m, m built from the bits O, O/2,
+// ..., O >> (NS - 1). While more than one value is live, a step keeps half of
+// them (the upper half on lanes whose bit O is set) and adds the partner lane's
+// copy of that half, so N values cost N - 1 shuffles instead of N * NS; once
+// one value is left the remaining steps are plain xor sums. On return
+// v[0 .. max(1, N >> NS)) hold the sums of the flat indices base, base + 1, ...,
+// and lanes that differ only in the bits of dup hold the same values.
+template <int C, int O, int NS, int N>
+__device__ __forceinline__ void xor_reduce(float (&v)[C], int lane, int& base, int& dup) {
+  if constexpr (NS > 0) {
+    if constexpr (N >= 2) {
+      constexpr int half = N / 2;
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = up ? v[i] : v[i + half];
+        const float keep = up ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      if (up) base += half;
+      xor_reduce<C, O / 2, NS - 1, half>(v, lane, base, dup);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      dup |= O;
+      xor_reduce<C, O / 2, NS - 1, 1>(v, lane, base, dup);
+    }
+  }
+}
+
+// grid (B * heads, n_chunks), K1 = K + 1 new rows per sequence. Three phases
+// over the chunk's positions:
+//   scores:  a half-warp reads one key (16 lanes x 8 dimensions, 256 contiguous
+//            bytes), every lane holding its 8 dimensions of all K1 queries in
+//            registers; the K1 dot products are summed over the half-warp by
+//            xor_reduce and written as pt[position][row];
+//   softmax: warp r takes row r: chunk max, exp, exp-sum (-> m, l);
+//   values:  warp w owns dimensions 16w .. 16w+15, its lanes split the
+//            positions 16 ways (16-byte value loads, the K1 weights of a
+//            position read as one or two 16-byte shared loads); the 16 partial
+//            sums are combined by xor_reduce at the end.
+template <int K1>
+__global__ void __launch_bounds__(kAttnThreads, 2) attn_chunk(const AttnArgs a) {
   griddep_launch_dependents();
   griddep_wait();
   constexpr int H = kAttnHeads * kAttnDim;
-  __shared__ float qs[kAttnMaxRows][kAttnDim];
-  __shared__ float ps[kAttnMaxRows][kAttnChunk];
-  __shared__ float red[kAttnThreads / 32];
-  __shared__ float mx[kAttnMaxRows], sm[kAttnMaxRows];
+  constexpr int KP = K1 <= 1 ? 1 : K1 <= 2 ? 2 : K1 <= 4 ? 4 : 8;  // rows padded to a power of two
+  constexpr int PW = 2 + kAttnDim;                                   // floats per row of a partial
+  static_assert(K1 >= 1 && K1 <= kAttnMaxRows && kAttnMaxRows <= 8 && kAttnThreads == 256 && kAttnDim == 128 &&
+                    kAttnChunk == 256,
+                "the lane maps below assume 8 warps, 128 dimensions, 256 positions, at most 8 rows");
+  __shared__ __align__(16) float pt[kAttnChunk][8];  // scores, then exp-weights: [position][row]
   const int b = blockIdx.x / kAttnHeads, h = blockIdx.x - b * kAttnHeads, c = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int L;
   const bool ok = attn_len_ok(a, b, &L);
-  const int visible = ok ? L + a.K1 : 0;  // positions any row of this step may see
+  const int visible = ok ? L + K1 : 0;  // positions any row of this step may see
   const int p0 = c * kAttnChunk, n = max(0, min(kAttnChunk, visible - p0));
-  float* part = a.part + (((size_t)b * kAttnHeads + h) * a.n_chunks + c) * a.K1 * (2 + kAttnDim);
+  float* part = a.part + (((size_t)b * kAttnHeads + h) * a.n_chunks + c) * K1 * PW;
   if (n == 0) {  // nothing here: an empty partial
-    for (int t = tid; t < a.K1; t += blockDim.x) {
-      part[(size_t)t * (2 + kAttnDim)] = -INFINITY;
-      part[(size_t)t * (2 + kAttnDim) + 1] = 0.0f;
+    for (int t = tid; t < K1; t += blockDim.x) {
+      part[(size_t)t * PW] = -INFINITY;
+      part[(size_t)t * PW + 1] = 0.0f;
     }
-    for (int t = tid; t < a.K1 * kAttnDim; t += blockDim.x)
-      part[(size_t)(t / kAttnDim) * (2 + kAttnDim) + 2 + t % kAttnDim] = 0.0f;
+    for (int t = tid; t < K1 * kAttnDim; t += blockDim.x) part[(size_t)(t / kAttnDim) * PW + 2 + t % kAttnDim] = 0.0f;
     return;
   }
-  for (int t = tid; t < a.K1 * kAttnDim; t += blockDim.x) {
-    const int r = t / kAttnDim, d = t - r * kAttnDim;
-    qs[r][d] = __bfloat162float(a.q[((size_t)b * a.K1 + r) * H + h * kAttnDim + d]);
-  }
-  __syncthreads();
   const float scale = 1.0f / sqrtf((float)kAttnDim);
-  // scores: thread = cache position p0 + tid
-  if (tid < n) {
-    const uint4* kp = reinterpret_cast<const uint4*>(a.cache + ((size_t)b * 2 * a.L_max + p0 + tid) * H + h * kAttnDim);
-    float acc[kAttnMaxRows];
+  {  // scores
+    const int dg = lane & 15, sub = lane >> 4;
+    float q[KP][8];
 #pragma unroll
-    for (int r = 0; r < kAttnMaxRows; ++r) acc[r] = 0.0f;
-#pragma unroll 4
-    for (int q8 = 0; q8 < kAttnDim / 8; ++q8) {
-      const uint4 v = __ldg(kp + q8);
-      const float kv[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                           bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-#pragma unroll
-      for (int r = 0; r < kAttnMaxRows; ++r) {
-        if (r < a.K1) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[r] = __fmaf_rn(qs[r][8 * q8 + e], kv[e], acc[r]);
-        }
-      }
+    for (int r = 0; r < KP; ++r) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (r < K1) u = *reinterpret_cast<const uint4*>(a.q + ((size_t)b * K1 + r) * H + h * kAttnDim + 8 * dg);
+      attn_unpack8(u, q[r]);
     }
-    const int pos = p0 + tid;
-    for (int r = 0; r < a.K1; ++r) ps[r][tid] = pos <= L + r ? acc[r] * scale : -INFINITY;  // causal
+    const __nv_bfloat16* kb = a.cache + ((size_t)b * 2 * a.L_max + p0) * H + h * kAttnDim + 8 * dg;
+#pragma unroll 8
+    for (int j = 0; j < kAttnChunk / 16; ++j) {
+      const int t = warp * (kAttnChunk / 8) + 2 * j + sub;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (t < n) u = __ldg(reinterpret_cast<const uint4*>(kb + (size_t)t * H));
+      float k8[8];
+      attn_unpack8(u, k8);
+      float sc[KP];
+#pragma unroll
+      for (int r = 0; r < KP; ++r) {
+        float d = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d = __fmaf_rn(q[r][e], k8[e], d);
+        sc[r] = d;
+      }
+      int r = 0, dup = 0;
+      xor_reduce<KP, 8, 4, KP>(sc, lane, r, dup);
+      if ((lane & dup) == 0 && r < K1 && t < n) pt[t][r] = p0 + t <= L + r ? sc[0] * scale : -INFINITY;  // causal
+    }
   }
-  for (int r = 0; r < a.K1; ++r)
-    if (tid >= n) ps[r][tid] = -INFINITY;
   __syncthreads();
-  // per row: max and exp-sum over the chunk
-  for (int r = 0; r < a.K1; ++r) {
-    float m = ps[r][tid];
+  if (warp < K1) {  // softmax statistics of row `warp` over the chunk
+    const int r = warp;
+    float v[kAttnChunk / 32];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kAttnChunk / 32; ++i) {
+      const int t = lane + 32 * i;
+      v[i] = t < n ? pt[t][r] : -INFINITY;
+      m = fmaxf(m, v[i]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-    if (tid == 0) {
-      float mm = red[0];
-      for (int w = 1; w < kAttnThreads / 32; ++w) mm = fmaxf(mm, red[w]);
-      mx[r] = mm;
+    float l = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kAttnChunk / 32; ++i) {
+      const int t = lane + 32 * i;
+      const float e = v[i] == -INFINITY ? 0.0f : expf(v[i] - m);
+      if (t < n) pt[t][r] = e;
+      l += e;
     }
-    __syncthreads();
-    const float e = ps[r][tid] == -INFINITY ? 0.0f : expf(ps[r][tid] - mx[r]);
-    ps[r][tid] = e;
-    float s = e;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    __syncthreads();
-    if (lane == 0) red[warp] = s;
-    __syncthreads();
-    if (tid == 0) {
-      float ss = 0.0f;
-      for (int w = 0; w < kAttnThreads / 32; ++w) ss += red[w];
-      sm[r] = ss;
-    }
-    __syncthreads();
-  }
-  // weighted values: thread = (dim, half of the rows)
-  const int d = tid & (kAttnDim - 1), half = tid >> 7;
-  float acc[kAttnMaxRows / 2];
-#pragma unroll
-  for (int j = 0; j < kAttnMaxRows / 2; ++j) acc[j] = 0.0f;
-  const __nv_bfloat16* vp = a.cache + ((size_t)(b * 2 + 1) * a.L_max + p0) * H + h * kAttnDim + d;
-  for (int t = 0; t < n; ++t) {
-    const float v = __bfloat162float(vp[(size_t)t * H]);
-#pragma unroll
-    for (int j = 0; j < kAttnMaxRows / 2; ++j) {
-      const int r = half + 2 * j;
-      if (r < a.K1) acc[j] = __fmaf_rn(ps[r][t], v, acc[j]);
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      part[(size_t)r * PW] = m;
+      part[(size_t)r * PW + 1] = l;
     }
   }
+  __syncthreads();
+  {  // exp-weighted values
+    const int dq = lane & 1, pg = lane >> 1;
+    const int d0 = 16 * warp + 8 * dq;
+    float acc[8 * KP];
 #pragma unroll
-  for (int j = 0; j < kAttnMaxRows / 2; ++j) {
-    const int r = half + 2 * j;
-    if (r < a.K1) part[(size_t)r * (2 + kAttnDim) + 2 + d] = acc[j];
-  }
-  if (tid < a.K1) {
-    part[(size_t)tid * (2 + kAttnDim)] = mx[tid];
-    part[(size_t)tid * (2 + kAttnDim) + 1] = sm[tid];
+    for (int i = 0; i < 8 * KP; ++i) acc[i] = 0.0f;
+    const __nv_bfloat16* vb = a.cache + ((size_t)(b * 2 + 1) * a.L_max + p0) * H + h * kAttnDim + d0;
+#pragma unroll 8
+    for (int i = 0; i < kAttnChunk / 16; ++i) {
+      const int t = pg + 16 * i;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      float4 pa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), pb = pa;
+      if (t < n) {
+        u = __ldg(reinterpret_cast<const uint4*>(vb + (size_t)t * H));
+        pa = *reinterpret_cast<const float4*>(&pt[t][0]);
+        if constexpr (KP > 4) pb = *reinterpret_cast<const float4*>(&pt[t][4]);
+      }
+      float v8[8];
+      attn_unpack8(u, v8);
+      const float p[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+      for (int r = 0; r < KP; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[r * 8 + e] = __fmaf_rn(p[r], v8[e], acc[r * 8 + e]);
+    }
+    int base = 0, dup = 0;
+    xor_reduce<8 * KP, 16, 4, 8 * KP>(acc, lane, base, dup);
+    constexpr int live = (8 * KP) >> 4 > 0 ? (8 * KP) >> 4 : 1;
+    if ((lane & dup) == 0) {
+#pragma unroll
+      for (int i = 0; i < live; ++i) {
+        const int f = base + i, r = f >> 3, e = f & 7;
+        if (r < K1) part[(size_t)r * PW + 2 + d0 + e] = acc[i];
+      }
+    }
   }
 }
 

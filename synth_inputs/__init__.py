@@ -40,6 +40,9 @@ TID_LM_HEAD = 4
 TID_DRAFTS = 5
 TID_HID = 6
 TID_EMB = 7  # token embedding of the synthetic decoder
+TID_ATTN_QKV = 8  # attention q/k/v projection
+TID_ATTN_O = 9  # attention output projection
+TID_KV = 10  # KV cache contents
 
 
 @dataclasses.dataclass(frozen=True)

@@ -66,3 +66,23 @@ def test_cache_overflow_is_reported_and_leaves_x(weights):
     assert st == 6, (st, info)
     assert np.array_equal(out[4:], x[4:])            # o = 0 for the overflowing sequence: out = x
     assert np.array_equal(new_cache[1], cache[1])    # and its cache is not written
+
+
+def test_attention_bench_shape(weights):
+    """The bench's attention launch (B = 32, K = 3, caches of 2,048 + 4
+    positions): every row against the oracle, half the sequences at the full
+    2,048 cached positions, the others ragged below it."""
+    B, K, L = 32, 3, 2048
+    lens = [L if b % 2 == 0 else L - 1 - (97 * b) % L for b in range(B)]
+    x, cache, out, new_cache, o = _run(weights, B, K, lens, L + K + 1, seed=2048)
+    st, info = vgv.vg_get_device_status()
+    assert st == 0, (st, info)
+    ref_out, ref_cache, mid = oracle.attn_verify(x, weights[0], weights[1], cache, lens, K)
+    assert row_rel_err(oracle.widen(o), oracle.widen(mid["o"])) <= ACT_TOL
+    assert row_rel_err(oracle.widen(out), oracle.widen(ref_out)) <= ACT_TOL
+    for b in (0, 1, B - 1):
+        L_b = lens[b]
+        assert np.array_equal(new_cache[b, :, :L_b], cache[b, :, :L_b])
+        for kv in (0, 1):
+            assert row_rel_err(oracle.widen(new_cache[b, kv, L_b: L_b + K + 1]),
+                               oracle.widen(ref_cache[b, kv, L_b: L_b + K + 1])) <= ACT_TOL
