@@ -35,6 +35,7 @@ EXPORTS = (
 # vg_kernel
 VG_KERNEL_ROUTER, VG_KERNEL_GROUPING, VG_KERNEL_EXPERTS = 0, 1, 2
 VG_KERNEL_COMBINE, VG_KERNEL_LM_HEAD, VG_KERNEL_ACCEPT = 3, 4, 5
+VG_KERNEL_ATTENTION = 6
 
 
 class VgError(RuntimeError):

@@ -12,7 +12,7 @@
 // attn_chunk: flash-decoding partials — one CTA per (sequence, head, chunk of
 //   kAttnChunk cache positions): the chunk's score max, exp-sum and
 //   exp-weighted value sum for each new row; every key and value of the chunk
-//   is read once for all K+1 rows.
+//   is read once for all K+1 rows, both products on the tensor cores.
 // attn_merge: merges a (sequence, head, row)'s chunk partials into o.
 // The projections run on the expert GEMM kernel (dense unit lists).
 #pragma once
@@ -75,171 +75,176 @@ __global__ void __launch_bounds__(256) attn_rope_append(const AttnArgs a) {
   vc[2 * pr + 1] = row[2 * H + 2 * pr + 1];
 }
 
-__device__ __forceinline__ void attn_unpack8(const uint4 u, float (&f)[8]) {
-  f[0] = bf16_lo(u.x), f[1] = bf16_hi(u.x), f[2] = bf16_lo(u.y), f[3] = bf16_hi(u.y);
-  f[4] = bf16_lo(u.z), f[5] = bf16_hi(u.z), f[6] = bf16_lo(u.w), f[7] = bf16_hi(u.w);
+// D += A B on the tensor cores, one m16n8k16 tile (bf16 operands, fp32
+// accumulators), A's rows 8..15 zero: a0 = A[g][2t, 2t+1], a2 = A[g][2t+8, 2t+9],
+// b0 = B[2t, 2t+1][g], b1 = B[2t+8, 2t+9][g], d = D[g][2t, 2t+1], D[g+8][2t, 2t+1]
+// with g = lane / 4, t = lane % 4.
+__device__ __forceinline__ void mma_16816_top(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
-// Sum of v[0 .. N) over the 2^NS lanes lane ^ m, m built from the bits O, O/2,
-// ..., O >> (NS - 1). While more than one value is live, a step keeps half of
-// them (the upper half on lanes whose bit O is set) and adds the partner lane's
-// copy of that half, so N values cost N - 1 shuffles instead of N * NS; once
-// one value is left the remaining steps are plain xor sums. On return
-// v[0 .. max(1, N >> NS)) hold the sums of the flat indices base, base + 1, ...,
-// and lanes that differ only in the bits of dup hold the same values.
-template <int C, int O, int NS, int N>
-__device__ __forceinline__ void xor_reduce(float (&v)[C], int lane, int& base, int& dup) {
-  if constexpr (NS > 0) {
-    if constexpr (N >= 2) {
-      constexpr int half = N / 2;
-      const bool up = (lane & O) != 0;
-#pragma unroll
-      for (int i = 0; i < half; ++i) {
-        const float send = up ? v[i] : v[i + half];
-        const float keep = up ? v[i + half] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
-      }
-      if (up) base += half;
-      xor_reduce<C, O / 2, NS - 1, half>(v, lane, base, dup);
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
-      dup |= O;
-      xor_reduce<C, O / 2, NS - 1, 1>(v, lane, base, dup);
-    }
-  }
+// Transpose of an 8 x 8 bf16 tile held one 32-bit pair per lane (lane (g, t)
+// holds row g, columns 2t, 2t+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  return d;
 }
 
-// grid (B * heads, n_chunks), K1 = K + 1 new rows per sequence. Three phases
-// over the chunk's positions:
-//   scores:  a half-warp reads one key (16 lanes x 8 dimensions, 256 contiguous
-//            bytes), every lane holding its 8 dimensions of all K1 queries in
-//            registers; the K1 dot products are summed over the half-warp by
-//            xor_reduce and written as pt[position][row];
-//   softmax: warp r takes row r: chunk max, exp, exp-sum (-> m, l);
-//   values:  warp w owns dimensions 16w .. 16w+15, its lanes split the
-//            positions 16 ways (16-byte value loads, the K1 weights of a
-//            position read as one or two 16-byte shared loads); the 16 partial
-//            sums are combined by xor_reduce at the end.
-template <int K1>
+// grid (B * heads, n_chunks), 256 threads; warp w takes positions 32w .. 32w+31
+// of the chunk, lane = (g, t) = (lane / 4, lane % 4), the K+1 <= 8 new rows as
+// rows 0..7 of 16-row tensor-core tiles (rows 8..15 zero).
+//   scores: S = Q K^T over 8 positions per tile; a lane loads 16 contiguous
+//     bytes (dimensions 32s + 8t .. +7 of one key, s = 0..3), giving the B
+//     operands of two k-steps; the queries are loaded with the same dimension
+//     order, so the contraction is unchanged;
+//   softmax over the warp's 32 positions, per row: max and the exp-weights,
+//     rounded to bf16 pairs that are already the A operand of the next product
+//     (the exp-sum is taken over the rounded weights);
+//   values: O += P V, 16 positions per k-step; a lane loads 16 contiguous bytes
+//     of a value row and movmatrix turns them into B operands, so lane (g, t)
+//     ends with dimensions 32s + 8t .. +7 of row g;
+//   the 8 warps' (max, exp-sum, values) are merged in shared memory into the
+//     chunk's partial.
 __global__ void __launch_bounds__(kAttnThreads, 2) attn_chunk(const AttnArgs a) {
   griddep_launch_dependents();
   griddep_wait();
   constexpr int H = kAttnHeads * kAttnDim;
-  constexpr int KP = K1 <= 1 ? 1 : K1 <= 2 ? 2 : K1 <= 4 ? 4 : 8;  // rows padded to a power of two
-  constexpr int PW = 2 + kAttnDim;                                   // floats per row of a partial
-  static_assert(K1 >= 1 && K1 <= kAttnMaxRows && kAttnMaxRows <= 8 && kAttnThreads == 256 && kAttnDim == 128 &&
-                    kAttnChunk == 256,
-                "the lane maps below assume 8 warps, 128 dimensions, 256 positions, at most 8 rows");
-  __shared__ __align__(16) float pt[kAttnChunk][8];  // scores, then exp-weights: [position][row]
+  constexpr int PW = 2 + kAttnDim;  // floats per row of a partial
+  constexpr int OW = kAttnDim + 4;  // padded row of the per-warp values
+  static_assert(kAttnMaxRows <= 8 && kAttnThreads == 256 && kAttnDim == 128 && kAttnChunk == 256,
+                "the lane maps below assume 8 warps of 32 positions, 128 dimensions, at most 8 rows");
+  __shared__ float wm[8][8], wl[8][8];              // per warp and row: max, exp-sum
+  __shared__ __align__(16) float wo[8][8][OW];      // per warp and row: exp-weighted values
   const int b = blockIdx.x / kAttnHeads, h = blockIdx.x - b * kAttnHeads, c = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int K1 = a.K1;
   int L;
   const bool ok = attn_len_ok(a, b, &L);
   const int visible = ok ? L + K1 : 0;  // positions any row of this step may see
   const int p0 = c * kAttnChunk, n = max(0, min(kAttnChunk, visible - p0));
   float* part = a.part + (((size_t)b * kAttnHeads + h) * a.n_chunks + c) * K1 * PW;
   if (n == 0) {  // nothing here: an empty partial
-    for (int t = tid; t < K1; t += blockDim.x) {
-      part[(size_t)t * PW] = -INFINITY;
-      part[(size_t)t * PW + 1] = 0.0f;
+    for (int i = tid; i < K1; i += blockDim.x) {
+      part[(size_t)i * PW] = -INFINITY;
+      part[(size_t)i * PW + 1] = 0.0f;
     }
-    for (int t = tid; t < K1 * kAttnDim; t += blockDim.x) part[(size_t)(t / kAttnDim) * PW + 2 + t % kAttnDim] = 0.0f;
+    for (int i = tid; i < K1 * kAttnDim; i += blockDim.x) part[(size_t)(i / kAttnDim) * PW + 2 + i % kAttnDim] = 0.0f;
     return;
   }
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  const int wp = 32 * warp;  // the warp's first position in the chunk
+  // ---- scores
+  uint4 qf[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s)
+    qf[s] = g < K1 ? *reinterpret_cast<const uint4*>(a.q + ((size_t)b * K1 + g) * H + h * kAttnDim + 32 * s + 8 * t)
+                   : zero4;
+  const __nv_bfloat16* kb = a.cache + ((size_t)b * 2 * a.L_max + p0 + wp) * H + h * kAttnDim + 8 * t;
+  float sc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int pos = 8 * j + g;  // the key this lane loads
+    uint4 kf[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      kf[s] = wp + pos < n ? __ldg(reinterpret_cast<const uint4*>(kb + (size_t)pos * H + 32 * s)) : zero4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[j][e] = 0.0f;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      mma_16816_top(sc[j], qf[s].x, qf[s].y, kf[s].x, kf[s].y);
+      mma_16816_top(sc[j], qf[s].z, qf[s].w, kf[s].z, kf[s].w);
+    }
+  }
+  // ---- softmax of row g over the warp's positions (lanes 4g .. 4g+3 share the row)
   const float scale = 1.0f / sqrtf((float)kAttnDim);
-  {  // scores
-    const int dg = lane & 15, sub = lane >> 4;
-    float q[KP][8];
+  float m = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < KP; ++r) {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (r < K1) u = *reinterpret_cast<const uint4*>(a.q + ((size_t)b * K1 + r) * H + h * kAttnDim + 8 * dg);
-      attn_unpack8(u, q[r]);
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int pos = wp + 8 * j + 2 * t + e;
+      const bool seen = g < K1 && pos < n && p0 + pos <= L + g;  // causal
+      sc[j][e] = seen ? sc[j][e] * scale : -INFINITY;
+      m = fmaxf(m, sc[j][e]);
     }
-    const __nv_bfloat16* kb = a.cache + ((size_t)b * 2 * a.L_max + p0) * H + h * kAttnDim + 8 * dg;
-#pragma unroll 8
-    for (int j = 0; j < kAttnChunk / 16; ++j) {
-      const int t = warp * (kAttnChunk / 8) + 2 * j + sub;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (t < n) u = __ldg(reinterpret_cast<const uint4*>(kb + (size_t)t * H));
-      float k8[8];
-      attn_unpack8(u, k8);
-      float sc[KP];
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  uint32_t pf[4];  // exp-weights of positions 8j + 2t, 8j + 2t + 1 as bf16 pairs
+  float l = 0.0f;
 #pragma unroll
-      for (int r = 0; r < KP; ++r) {
-        float d = 0.0f;
+  for (int j = 0; j < 4; ++j) {
+    const float e0 = sc[j][0] == -INFINITY ? 0.0f : expf(sc[j][0] - m);
+    const float e1 = sc[j][1] == -INFINITY ? 0.0f : expf(sc[j][1] - m);
+    const __nv_bfloat162 pp = __floats2bfloat162_rn(e0, e1);
+    pf[j] = *reinterpret_cast<const uint32_t*>(&pp);
+    l += __low2float(pp) + __high2float(pp);
+  }
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  // ---- values: O = P V over the warp's positions, two k-steps of 16
+  float o[4][4][4];  // [dimension block s][tile j][accumulator]: row g, dimensions 32s + 8t + 2j + {0, 1}
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d = __fmaf_rn(q[r][e], k8[e], d);
-        sc[r] = d;
-      }
-      int r = 0, dup = 0;
-      xor_reduce<KP, 8, 4, KP>(sc, lane, r, dup);
-      if ((lane & dup) == 0 && r < K1 && t < n) pt[t][r] = p0 + t <= L + r ? sc[0] * scale : -INFINITY;  // causal
+  for (int s = 0; s < 4; ++s)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[s][j][e] = 0.0f;
+  const __nv_bfloat16* vb = a.cache + ((size_t)(b * 2 + 1) * a.L_max + p0 + wp) * H + h * kAttnDim + 8 * t;
+#pragma unroll
+  for (int kp = 0; kp < 2; ++kp) {
+    const int lo = 16 * kp + g, hi = lo + 8;  // the value rows this lane loads
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint4 vl = wp + lo < n ? __ldg(reinterpret_cast<const uint4*>(vb + (size_t)lo * H + 32 * s)) : zero4;
+      const uint4 vh = wp + hi < n ? __ldg(reinterpret_cast<const uint4*>(vb + (size_t)hi * H + 32 * s)) : zero4;
+      const uint32_t rl[4] = {vl.x, vl.y, vl.z, vl.w}, rh[4] = {vh.x, vh.y, vh.z, vh.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        mma_16816_top(o[s][j], pf[2 * kp], pf[2 * kp + 1], movmatrix_trans(rl[j]), movmatrix_trans(rh[j]));
     }
   }
-  __syncthreads();
-  if (warp < K1) {  // softmax statistics of row `warp` over the chunk
-    const int r = warp;
-    float v[kAttnChunk / 32];
-    float m = -INFINITY;
+  // ---- merge the 8 warps into the chunk's partial
+  if (t == 0) {
+    wm[warp][g] = m;
+    wl[warp][g] = l;
+  }
 #pragma unroll
-    for (int i = 0; i < kAttnChunk / 32; ++i) {
-      const int t = lane + 32 * i;
-      v[i] = t < n ? pt[t][r] : -INFINITY;
-      m = fmaxf(m, v[i]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kAttnChunk / 32; ++i) {
-      const int t = lane + 32 * i;
-      const float e = v[i] == -INFINITY ? 0.0f : expf(v[i] - m);
-      if (t < n) pt[t][r] = e;
-      l += e;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      part[(size_t)r * PW] = m;
-      part[(size_t)r * PW + 1] = l;
-    }
+  for (int s = 0; s < 4; ++s) {
+    float* dst = &wo[warp][g][32 * s + 8 * t];
+    *reinterpret_cast<float4*>(dst) = make_float4(o[s][0][0], o[s][0][1], o[s][1][0], o[s][1][1]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(o[s][2][0], o[s][2][1], o[s][3][0], o[s][3][1]);
   }
   __syncthreads();
-  {  // exp-weighted values
-    const int dq = lane & 1, pg = lane >> 1;
-    const int d0 = 16 * warp + 8 * dq;
-    float acc[8 * KP];
+  for (int i = tid; i < K1 * (kAttnDim / 4); i += kAttnThreads) {
+    const int r = i / (kAttnDim / 4), d4 = 4 * (i % (kAttnDim / 4));
+    float mm = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 8 * KP; ++i) acc[i] = 0.0f;
-    const __nv_bfloat16* vb = a.cache + ((size_t)(b * 2 + 1) * a.L_max + p0) * H + h * kAttnDim + d0;
-#pragma unroll 8
-    for (int i = 0; i < kAttnChunk / 16; ++i) {
-      const int t = pg + 16 * i;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      float4 pa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), pb = pa;
-      if (t < n) {
-        u = __ldg(reinterpret_cast<const uint4*>(vb + (size_t)t * H));
-        pa = *reinterpret_cast<const float4*>(&pt[t][0]);
-        if constexpr (KP > 4) pb = *reinterpret_cast<const float4*>(&pt[t][4]);
-      }
-      float v8[8];
-      attn_unpack8(u, v8);
-      const float p[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, wm[w][r]);
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float ls = 0.0f;
 #pragma unroll
-      for (int r = 0; r < KP; ++r)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r * 8 + e] = __fmaf_rn(p[r], v8[e], acc[r * 8 + e]);
+    for (int w = 0; w < 8; ++w) {
+      if (wm[w][r] == -INFINITY) continue;  // no visible position in that warp's share
+      const float f = expf(wm[w][r] - mm);
+      ls = __fmaf_rn(wl[w][r], f, ls);
+      const float4 v = *reinterpret_cast<const float4*>(&wo[w][r][d4]);
+      acc.x = __fmaf_rn(v.x, f, acc.x);
+      acc.y = __fmaf_rn(v.y, f, acc.y);
+      acc.z = __fmaf_rn(v.z, f, acc.z);
+      acc.w = __fmaf_rn(v.w, f, acc.w);
     }
-    int base = 0, dup = 0;
-    xor_reduce<8 * KP, 16, 4, 8 * KP>(acc, lane, base, dup);
-    constexpr int live = (8 * KP) >> 4 > 0 ? (8 * KP) >> 4 : 1;
-    if ((lane & dup) == 0) {
-#pragma unroll
-      for (int i = 0; i < live; ++i) {
-        const int f = base + i, r = f >> 3, e = f & 7;
-        if (r < K1) part[(size_t)r * PW + 2 + d0 + e] = acc[i];
-      }
+    float* pr = part + (size_t)r * PW;
+    pr[2 + d4] = acc.x;
+    pr[3 + d4] = acc.y;
+    pr[4 + d4] = acc.z;
+    pr[5 + d4] = acc.w;
+    if (d4 == 0) {
+      pr[0] = mm;
+      pr[1] = ls;
     }
   }
 }

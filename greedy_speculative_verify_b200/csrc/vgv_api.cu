@@ -1010,18 +1010,10 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  void (*chunk)(const AttnArgs) = nullptr;
-  switch (K + 1) {
-    case 1: chunk = attn_chunk<1>; break;
-    case 2: chunk = attn_chunk<2>; break;
-    case 3: chunk = attn_chunk<3>; break;
-    case 4: chunk = attn_chunk<4>; break;
-    case 5: chunk = attn_chunk<5>; break;
-    case 6: chunk = attn_chunk<6>; break;
-    case 7: chunk = attn_chunk<7>; break;
-    default: chunk = attn_chunk<8>; break;  // K + 1 <= kAttnMaxRows = 8 was checked above
+  {
+    ProfScope ps(VG_KERNEL_ATTENTION, s);
+    if (cudaLaunchKernelEx(&cfg, attn_chunk, a) != cudaSuccess) return cuda_fail();
   }
-  if (cudaLaunchKernelEx(&cfg, chunk, a) != cudaSuccess) return cuda_fail();
   if (launch_dep(attn_merge, B * kAttnHeads * (K + 1), kAttnDim, 0, s, Launch::kPlain, a) != cudaSuccess)
     return cuda_fail();
   // out = x + W_o o

@@ -179,7 +179,9 @@ typedef enum vg_kernel {
                               layer's own output, or the stack's last layer) */
   VG_KERNEL_LM_HEAD = 4,   /* LM-head GEMM + per-tile argmax */
   VG_KERNEL_ACCEPT = 5,    /* argmax reduction + prefix accept */
-  VG_KERNEL_KINDS = 6
+  VG_KERNEL_ATTENTION = 6, /* verifier attention: the chunk partials (scores,
+                              softmax, values) of vg_attn_verify */
+  VG_KERNEL_KINDS = 7
 } vg_kernel;
 
 /* Same object as cudaEvent_t. */
