@@ -973,7 +973,11 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
       !aligned16(o_out))
     return VG_ERR_INVALID_ARG;
   const int R = B * (K + 1);
-  if (overlaps(x, (size_t)R * kH * 2, out, (size_t)R * kH * 2)) return VG_ERR_INVALID_ARG;
+  const size_t rows_bytes = (size_t)R * kH * 2, cache_bytes = (size_t)B * 2 * L_max * kH * 2;
+  if (overlaps(x, rows_bytes, out, rows_bytes) || overlaps(kv_cache, cache_bytes, out, rows_bytes)) return VG_ERR_INVALID_ARG;
+  if (o_out && (overlaps(x, rows_bytes, o_out, rows_bytes) || overlaps(out, rows_bytes, o_out, rows_bytes) ||
+                overlaps(kv_cache, cache_bytes, o_out, rows_bytes)))
+    return VG_ERR_INVALID_ARG;
   const AttnWs L = attn_layout(B, K, L_max);
   if (workspace == nullptr || workspace_bytes < L.total) return VG_ERR_WORKSPACE;
   DevState* dev = nullptr;

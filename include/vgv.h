@@ -364,8 +364,13 @@ vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void
  * is read, not advanced (advance it by the committed tokens; a later step
  * overwrites the positions of rejected drafts). K+1 <= 8, L_max <= 32768;
  * lens[b] + K + 1 > L_max records VG_ERR_DEVICE_BOUNDS and gives o = 0 for that
- * sequence. out must not overlap x. o_out, if not NULL, bf16 [B*(K+1), H]
- * receives the heads' output o before the output projection. Errors: VG_ERR_INVALID_ARG,
+ * sequence. o_out, if not NULL, bf16 [B*(K+1), H] receives the heads' output o
+ * before the output projection. All pointers are device memory, the arrays
+ * 16-byte aligned; out and o_out must not overlap x or each other, and none of
+ * them kv_cache. Precision: both products of a head (q.k and the
+ * probability-weighted sum of v) run on the tensor cores with bf16 operands and
+ * fp32 accumulation, so the softmax weights enter the second product rounded to
+ * bf16 (their sum is taken over the rounded weights). Errors: VG_ERR_INVALID_ARG,
  * VG_ERR_WORKSPACE, VG_ERR_CUDA.
  * ------------------------------------------------------------------------- */
 size_t vg_attn_workspace_bytes(int32_t B, int32_t K, int32_t L_max);

@@ -172,4 +172,9 @@ def test_attention_validation_before_launch(lib):
     assert f(*args(x=None)) == 1
     assert f(*args(out=A + 64)) == 1              # out overlaps x
     assert f(*args(wq=A + 8)) == 1                # misaligned weights
+    assert f(*args(out=A + (3 << 30) + 4096)) == 1  # out inside the cache
+    assert f(*args(o=A + 64)) == 1                # o_out overlaps x
+    assert f(*args(o=A + (5 << 30))) == 1         # o_out overlaps out
+    assert f(*args(o=A + (3 << 30))) == 1         # o_out inside the cache
+    assert f(*args(o=A + (7 << 30) + 8)) == 1     # misaligned o_out
     assert f(*args(n=need - 1)) == 3
