@@ -86,3 +86,22 @@ def test_attention_bench_shape(weights):
         for kv in (0, 1):
             assert row_rel_err(oracle.widen(new_cache[b, kv, L_b: L_b + K + 1]),
                                oracle.widen(ref_cache[b, kv, L_b: L_b + K + 1])) <= ACT_TOL
+
+
+def test_attention_longest_cache(weights):
+    """The largest cache the call takes (L_max = 32,768 positions, the decoder's
+    position limit) with the most new rows (K = 7): one sequence filling it to
+    the last position, one nearly empty."""
+    B, K, L_max = 2, 7, 32768
+    lens = [L_max - K - 1, 5]
+    x, cache, out, new_cache, o = _run(weights, B, K, lens, L_max, seed=32768)
+    st, info = vgv.vg_get_device_status()
+    assert st == 0, (st, info)
+    ref_out, ref_cache, mid = oracle.attn_verify(x, weights[0], weights[1], cache, lens, K)
+    assert row_rel_err(oracle.widen(o), oracle.widen(mid["o"])) <= ACT_TOL
+    assert row_rel_err(oracle.widen(out), oracle.widen(ref_out)) <= ACT_TOL
+    for b, L in enumerate(lens):
+        for kv in (0, 1):
+            assert row_rel_err(oracle.widen(new_cache[b, kv, L: L + K + 1]),
+                               oracle.widen(ref_cache[b, kv, L: L + K + 1])) <= ACT_TOL
+    assert np.array_equal(new_cache[0, :, :lens[0]], cache[0, :, :lens[0]])
