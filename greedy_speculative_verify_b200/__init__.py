@@ -290,7 +290,10 @@ def vg_attn_workspace_bytes(B, K, L_max):
 
 
 def vg_attn_verify(B, K, x, w_qkv, w_o, kv_cache, lens, out, workspace, o_out=None, stream=None):
-    """One attention layer of a verify step; kv_cache [B, 2, L_max, H]."""
+    """One attention layer of a verify step; kv_cache [B, 2, L_max, H] (its
+    third dimension is passed as L_max, so it must be that dense shape)."""
+    if kv_cache.dim() != 4 or kv_cache.shape[0] != B or kv_cache.shape[1] != 2 or not kv_cache.is_contiguous():
+        raise ValueError("kv_cache must be a contiguous [B, 2, L_max, H] tensor")
     _check(load().vg_attn_verify(B, K, kv_cache.shape[2], _ptr(x), _ptr(w_qkv), _ptr(w_o), _ptr(kv_cache), _ptr(lens),
                                  _ptr(out), _ptr(o_out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "vg_attn_verify")

@@ -178,3 +178,16 @@ def test_attention_validation_before_launch(lib):
     assert f(*args(o=A + (3 << 30))) == 1         # o_out inside the cache
     assert f(*args(o=A + (7 << 30) + 8)) == 1     # misaligned o_out
     assert f(*args(n=need - 1)) == 3
+
+
+def test_attention_binding_checks_cache_shape():
+    """The binding passes the cache's third dimension as L_max, so it refuses a
+    cache that is not a dense [B, 2, L_max, H] tensor before any library call."""
+    import torch
+
+    good = torch.zeros(2, 2, 16, 1280, dtype=torch.bfloat16)
+    for bad in (torch.zeros(3, 2, 16, 1280, dtype=torch.bfloat16),       # wrong B
+                torch.zeros(2, 16, 1280, dtype=torch.bfloat16),          # not 4-d
+                good.transpose(2, 3)):                                    # not dense
+        with pytest.raises(ValueError):
+            vgv.vg_attn_verify(2, 3, None, None, None, bad, None, None, None)
