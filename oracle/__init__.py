@@ -22,7 +22,7 @@ What the pages fix, and where each piece comes from:
   (jina.ai/de), section "Modell und Training"; the same page, section
   "Spekulatives Decoding auf einer L4", counts the bonus token in tau.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent (each one a choice of this oracle, stated here):
 
 * router logits are four fp32 fused-multiply-add chains over the contiguous
   quarters of h (each from +0, increasing h), combined as (q0+q1)+(q2+q3) in

@@ -5,7 +5,7 @@ token, plus two shared experts that every token visits ("Jina AI's 3.4B OCR mode
 targets faster page parsing", section "A compressed visual front end"); 12
 decoder layers, hidden 1280 (jina-ocr-v1 model card, architecture paragraph).
 The expert form (SwiGLU), the width I = 896, unweighted shared experts and the
-residual add are readings, listed in the design doc.
+residual add are readings of the pages, not facts they state.
 
 Each expert's bf16 weights are one contiguous block gate [I,H] | up [I,H] |
 down [H,I], row-major.

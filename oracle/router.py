@@ -4,7 +4,7 @@ Test infrastructure only. The pages state that top-6 routing picks six of the 64
 routed experts for every token ("Jina AI's 3.4B OCR model targets faster page
 parsing", section "A compressed visual front end"; jina-ocr-v1 model card,
 architecture paragraph). They give no formula; the readings below are the
-plainest ones and are listed in the design doc.
+plainest ones consistent with the rest of the pages.
 """
 import numpy as np
 
