@@ -35,7 +35,7 @@ def _rank_main(rank, world, port, out):
 
 def test_aggregate_over_two_gloo_ranks():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of a threaded process
     mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
         assert out[r] == (2.0, 10.0, 300)  # max, max, sum on every rank
