@@ -14,7 +14,9 @@
 //   exp-weighted value sum for each new row; every key and value of the chunk
 //   is read once for all K+1 rows, both products on the tensor cores.
 // attn_merge: merges a (sequence, head, row)'s chunk partials into o.
-// The projections run on the expert GEMM kernel (dense unit lists).
+// attn_proj_splitk: the q/k/v and output projections as fp32 partial sums over
+//   256-wide slices of the reduction, summed in a fixed order by their readers
+//   (attn_rope_append, attn_residual), which round the sum to bf16.
 #pragma once
 #include "common.cuh"
 
@@ -24,11 +26,13 @@ constexpr int kAttnHeads = 10, kAttnDim = 128;
 constexpr int kAttnChunk = 256;   // cache positions per CTA
 constexpr int kAttnMaxRows = 8;   // K + 1 <= 8 new rows per sequence
 constexpr int kAttnThreads = 256;
+constexpr int kProjN = 64, kProjK = 256, kProjM = 128;  // projection block: outputs, reduction slice, rows
 
 struct AttnArgs {
   int32_t B, K1, L_max;          // K1 = K + 1 rows per sequence
   const int32_t* lens;           // [B] cached positions before this step
-  const __nv_bfloat16* qkv;      // [B*K1, 3H]
+  const float* qkv_part;         // [splits, B*K1, 3H] fp32 partial sums of x W_qkv^T
+  int32_t splits;
   __nv_bfloat16* q;              // [B*K1, H] rotated queries
   __nv_bfloat16* cache;          // [B, 2, L_max, H]
   float* part;                   // [B, heads, n_chunks, K1, 2 + dim]: m, l, acc
@@ -39,6 +43,91 @@ struct AttnArgs {
 __device__ __forceinline__ bool attn_len_ok(const AttnArgs& a, int b, int* L) {
   *L = a.lens[b];
   return *L >= 0 && *L + a.K1 <= a.L_max;
+}
+
+// D += A B on the tensor cores, one m16n8k16 tile (bf16 operands, fp32
+// accumulators), g = lane / 4, t = lane % 4: a0 = A[g][2t, 2t+1],
+// a1 = A[g+8][2t, 2t+1], a2 = A[g][2t+8, 2t+9], a3 = A[g+8][2t+8, 2t+9],
+// b0 = B[2t, 2t+1][g], b1 = B[2t+8, 2t+9][g], d = D[g][2t, 2t+1], D[g+8][2t, 2t+1].
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// part[s][r][n] = sum over k in [256 s, 256 s + 256) of x[r][k] W[n][k] (fp32),
+// for x bf16 [R, K] and W bf16 [N, K] (N a multiple of 64, K of 256).
+// grid (N / 64, K / 256, cdiv(R, 128)), 256 threads: warp w takes rows
+// 128 z + 16 w .. +15 against the block's 64 outputs (8 tensor-core n-tiles).
+// A lane loads 16 contiguous bytes of a row of x and of W per 32-wide step of
+// the reduction; both operands take the same order of k inside the step, so
+// the sum is unchanged. The reduction is split so that a launch has
+// N / 64 x K / 256 blocks streaming the weights (60 x 5 for q/k/v).
+__global__ void __launch_bounds__(256) attn_proj_splitk(const __nv_bfloat16* __restrict__ x,
+                                                        const __nv_bfloat16* __restrict__ w, int R, int N, int K,
+                                                        float* __restrict__ part) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int n0 = blockIdx.x * kProjN, sl = blockIdx.y, k0 = sl * kProjK;
+  const int r0 = blockIdx.z * kProjM + 16 * warp;
+  if (r0 >= R) return;  // the whole warp: rows past the end
+  const int ra = r0 + g, rb = r0 + g + 8;
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  const __nv_bfloat16* xa = x + (size_t)ra * K + k0 + 8 * t;
+  const __nv_bfloat16* xb = x + (size_t)rb * K + k0 + 8 * t;
+  const __nv_bfloat16* wr = w + (size_t)(n0 + g) * K + k0 + 8 * t;
+  float acc[kProjN / 8][4];
+#pragma unroll
+  for (int j = 0; j < kProjN / 8; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
+#pragma unroll 2
+  for (int q = 0; q < kProjK / 32; ++q) {
+    const uint4 av = ra < R ? __ldg(reinterpret_cast<const uint4*>(xa + 32 * q)) : zero4;
+    const uint4 bv = rb < R ? __ldg(reinterpret_cast<const uint4*>(xb + 32 * q)) : zero4;
+#pragma unroll
+    for (int j = 0; j < kProjN / 8; ++j) {
+      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + (size_t)8 * j * K + 32 * q));
+      mma_16816(acc[j], av.x, bv.x, av.y, bv.y, wv.x, wv.y);
+      mma_16816(acc[j], av.z, bv.z, av.w, bv.w, wv.z, wv.w);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kProjN / 8; ++j) {
+    const int n = n0 + 8 * j + 2 * t;
+    if (ra < R) *reinterpret_cast<float2*>(part + ((size_t)sl * R + ra) * N + n) = make_float2(acc[j][0], acc[j][1]);
+    if (rb < R) *reinterpret_cast<float2*>(part + ((size_t)sl * R + rb) * N + n) = make_float2(acc[j][2], acc[j][3]);
+  }
+}
+
+// bf16 of the fixed-order sum of `splits` partials p[0], p[stride], ...
+__device__ __forceinline__ float proj_sum_bf16(const float* p, int splits, size_t stride) {
+  float v = 0.0f;
+  for (int s = 0; s < splits; ++s) v += p[(size_t)s * stride];
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// out = bf16(x + bf16(sum_s part[s])), four elements per thread (n a multiple of 4).
+__global__ void __launch_bounds__(256) attn_residual(const __nv_bfloat16* __restrict__ x,
+                                                     const float* __restrict__ part, int splits, int n,
+                                                     __nv_bfloat16* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= n / 4) return;
+  float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int s = 0; s < splits; ++s) {
+    const float4 p = reinterpret_cast<const float4*>(part + (size_t)s * n)[c];
+    v.x += p.x, v.y += p.y, v.z += p.z, v.w += p.w;
+  }
+  const uint2 xv = reinterpret_cast<const uint2*>(x)[c];
+  const float y0 = __bfloat162float(__float2bfloat16_rn(v.x)), y1 = __bfloat162float(__float2bfloat16_rn(v.y));
+  const float y2 = __bfloat162float(__float2bfloat16_rn(v.z)), y3 = __bfloat162float(__float2bfloat16_rn(v.w));
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(bf16_lo(xv.x) + y0, bf16_hi(xv.x) + y1);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(bf16_lo(xv.y) + y2, bf16_hi(xv.y) + y3);
+  reinterpret_cast<uint2*>(out)[c] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
 }
 
 // One thread per (row, pair) of q and of k.
@@ -60,19 +149,22 @@ __global__ void __launch_bounds__(256) attn_rope_append(const AttnArgs a) {
   const double ang = (double)(L + i) * pow(10000.0, -2.0 * j / kAttnDim);
   double sn, cs;
   sincos(ang, &sn, &cs);
-  const __nv_bfloat16* row = a.qkv + (size_t)r * 3 * H;
-  auto turn = [&](const __nv_bfloat16* src, __nv_bfloat16* dst) {
-    const float x0 = __bfloat162float(src[2 * pr]), x1 = __bfloat162float(src[2 * pr + 1]);
+  const size_t stride = (size_t)R * 3 * H;  // one partial of the projection
+  const float* row = a.qkv_part + (size_t)r * 3 * H;
+  // q, k, v = bf16 of the projection (the sum of its partials)
+  auto val = [&](int col) { return proj_sum_bf16(row + col, a.splits, stride); };
+  auto turn = [&](int col, __nv_bfloat16* dst) {
+    const float x0 = val(col + 2 * pr), x1 = val(col + 2 * pr + 1);
     const double y0 = (double)x0 * cs - (double)x1 * sn, y1 = (double)x0 * sn + (double)x1 * cs;
     dst[2 * pr] = __float2bfloat16_rn((float)y0);
     dst[2 * pr + 1] = __float2bfloat16_rn((float)y1);
   };
-  turn(row, a.q + (size_t)r * H);
+  turn(0, a.q + (size_t)r * H);
   __nv_bfloat16* kc = a.cache + ((size_t)b * 2 * a.L_max + (L + i)) * H;
   __nv_bfloat16* vc = a.cache + ((size_t)(b * 2 + 1) * a.L_max + (L + i)) * H;
-  turn(row + H, kc);
-  vc[2 * pr] = row[2 * H + 2 * pr];
-  vc[2 * pr + 1] = row[2 * H + 2 * pr + 1];
+  turn(H, kc);
+  vc[2 * pr] = __float2bfloat16_rn(val(2 * H + 2 * pr));
+  vc[2 * pr + 1] = __float2bfloat16_rn(val(2 * H + 2 * pr + 1));
 }
 
 // D += A B on the tensor cores, one m16n8k16 tile (bf16 operands, fp32

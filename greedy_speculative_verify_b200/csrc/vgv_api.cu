@@ -934,8 +934,9 @@ extern "C" vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w,
 // ------------------------------------------------------------ verifier attention
 namespace {
 struct AttnWs {
-  size_t qkv, q, o, proj, part, sched, zero, total;
+  size_t pk, q, o, part, total;
 };
+constexpr int kProjSplits = kH / vg::kProjK;  // partial sums of a projection (5)
 AttnWs attn_layout(int B, int K, int L_max) {
   const size_t R = (size_t)B * (K + 1);
   AttnWs L{};
@@ -945,13 +946,10 @@ AttnWs attn_layout(int B, int K, int L_max) {
     off = align256(off + bytes);
     return o;
   };
-  L.qkv = take(R * 3 * kH * 2);
+  L.pk = take((size_t)kProjSplits * R * 3 * kH * 4);  // projection partials (q/k/v, then the output's)
   L.q = take(R * kH * 2);
   L.o = take(R * kH * 2);
-  L.proj = take(R * kH * 2);
   L.part = take((size_t)B * vg::kAttnHeads * vg::cdiv(L_max, vg::kAttnChunk) * (K + 1) * (2 + vg::kAttnDim) * 4);
-  L.sched = take((size_t)(2 + vg::cdiv((int)R, 16)) * 4);
-  L.zero = take(16);
   L.total = off;
   return L;
 }
@@ -986,18 +984,30 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(ws + o); };
-  auto i32 = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
-  if (cudaMemsetAsync(ws + L.zero, 0, 16, s) != cudaSuccess) return cuda_fail();
-  // qkv = x W_qkv^T: a down-only unit list with 3H output rows
-  if ((st = launch_dense(dev, R, w_qkv, false, kH, 3 * kH, nullptr, const_cast<void*>(x), bf(L.qkv), i32(L.sched),
-                         i32(L.zero), s)) != VG_OK)
-    return st;
+  float* pk = reinterpret_cast<float*>(ws + L.pk);
+  const int mblocks = cdiv(R, kProjM);
+  auto launch_proj = [&](const void* act, const void* wgt, int n_out) {
+    cudaLaunchConfig_t pc = {};  // 3-d grid: (64 outputs, 256-wide reduction slice, 128 rows)
+    pc.gridDim = dim3(n_out / kProjN, kProjSplits, mblocks);
+    pc.blockDim = dim3(256);
+    pc.stream = s;
+    cudaLaunchAttribute pa[1];
+    pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pa[0].val.programmaticStreamSerializationAllowed = 1;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    return cudaLaunchKernelEx(&pc, attn_proj_splitk, static_cast<const __nv_bfloat16*>(act),
+                              static_cast<const __nv_bfloat16*>(wgt), R, n_out, (int)kH, pk);
+  };
+  // q/k/v = x W_qkv^T as split partial sums
+  if (launch_proj(x, w_qkv, 3 * kH) != cudaSuccess) return cuda_fail();
   AttnArgs a{};
   a.B = B;
   a.K1 = K + 1;
   a.L_max = L_max;
   a.lens = lens;
-  a.qkv = bf(L.qkv);
+  a.qkv_part = pk;
+  a.splits = kProjSplits;
   a.q = bf(L.q);
   a.cache = static_cast<__nv_bfloat16*>(kv_cache);
   a.part = reinterpret_cast<float*>(ws + L.part);
@@ -1020,12 +1030,10 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   }
   if (launch_dep(attn_merge, B * kAttnHeads * (K + 1), kAttnDim, 0, s, Launch::kPlain, a) != cudaSuccess)
     return cuda_fail();
-  // out = x + W_o o
-  if ((st = launch_dense(dev, R, w_o, false, kH, kH, nullptr, a.o, bf(L.proj), i32(L.sched), i32(L.zero), s)) !=
-      VG_OK)
-    return st;
-  if (launch_dep(mtp_residual, cdiv(R * kH / 8, 256), 256, 0, s, Launch::kPlain, static_cast<const __nv_bfloat16*>(x),
-                 (const __nv_bfloat16*)bf(L.proj), R * kH, static_cast<__nv_bfloat16*>(out)) != cudaSuccess)
+  // out = x + W_o o: split partials (over the q/k/v partials, consumed by now), then the residual
+  if (launch_proj(a.o, w_o, kH) != cudaSuccess) return cuda_fail();
+  if (launch_dep(attn_residual, cdiv(R * kH / 4, 256), 256, 0, s, Launch::kPlain, static_cast<const __nv_bfloat16*>(x),
+                 (const float*)pk, kProjSplits, R * kH, static_cast<__nv_bfloat16*>(out)) != cudaSuccess)
     return cuda_fail();
   return VG_OK;
 }
