@@ -167,14 +167,9 @@ __global__ void __launch_bounds__(256) attn_rope_append(const AttnArgs a) {
   vc[2 * pr + 1] = __float2bfloat16_rn(val(2 * H + 2 * pr + 1));
 }
 
-// D += A B on the tensor cores, one m16n8k16 tile (bf16 operands, fp32
-// accumulators), A's rows 8..15 zero: a0 = A[g][2t, 2t+1], a2 = A[g][2t+8, 2t+9],
-// b0 = B[2t, 2t+1][g], b1 = B[2t+8, 2t+9][g], d = D[g][2t, 2t+1], D[g+8][2t, 2t+1]
-// with g = lane / 4, t = lane % 4.
+// mma_16816 with A's rows 8..15 zero (the K+1 <= 8 new rows in a 16-row tile).
 __device__ __forceinline__ void mma_16816_top(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+  mma_16816(d, a0, 0u, a2, 0u, b0, b1);
 }
 
 // Transpose of an 8 x 8 bf16 tile held one 32-bit pair per lane (lane (g, t)
