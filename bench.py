@@ -49,10 +49,32 @@ WORKLOAD = {
     "l2": "inputs larger than L2: 5.78 GB of weights per step vs 126 MB L2, no flush",
 }
 EXPERT_W_BYTES = 3 * I * H * 2  # gate + up + down of one expert, bf16 (6,881,280 B)
-# DRAM bytes (read + write) of one expert-GEMM launch at 128 tokens, from one
-# ncu capture of that kernel (456.5 MB read + 5.1 MB written); to be re-taken
-# whenever that kernel changes
-EXPERT_TRAFFIC_BYTES = 461.6e6
+ROUTER_W_BYTES = E * H * 2      # 163,840 B per layer
+LM_HEAD_BYTES = V * H * 2       # 330,956,800 B
+NOMINAL_HBM_GBS = 8000.0        # "about 8 TB/s", the nominal figure the decode target is stated on
+# DRAM bytes (read + write) of one expert-GEMM launch at 128 tokens from one ncu
+# capture, with the SHA-256 (first 16 hex digits) of the kernel source it was
+# taken on; the bench reports it only while the source is unchanged.
+EXPERT_TRAFFIC = {"bytes": 461.6e6, "source": "greedy_speculative_verify_b200/csrc/gemm_moe.cuh",
+                  "source_sha16": "74156f6761b3f862", "profile": "profiles/moe_expert_gemms_t128.md"}
+
+
+def _traffic(rec):
+    import hashlib
+
+    try:
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return rec["bytes"] if sha == rec["source_sha16"] else None
+
+
+def step_weight_bytes(n_touched):
+    """Algorithmic bytes of one decode verify step: per layer the router, the two
+    shared experts and every touched routed expert, once; then the LM head.
+    Activations are not counted (reported separately)."""
+    return sum(ROUTER_W_BYTES + (n + S) * EXPERT_W_BYTES for n in n_touched) + LM_HEAD_BYTES
 
 
 def _env():
@@ -138,6 +160,119 @@ def measure_prefill(vgv, si, dev, reps=10):
             "frac_layer": PREFILL_FLOP / (layer_ms / 1e3) / 1e12 / peak,
             "frac_expert_gemms": gemm_flop / (gemm_ms / 1e3) / 1e12 / peak,
             "breakdown_ms": {n: min(v) for n, v in parts.items()}}
+
+
+SKEW_T = 4096
+SKEW_FLOP = 2 * TOPK * SKEW_T * 3 * I * H + 2 * S * SKEW_T * 3 * I * H + 2 * SKEW_T * E * H
+SKEW_B, SKEW_K = 2048, 1
+SKEW_LM_FLOP = 2 * SKEW_B * (SKEW_K + 1) * V * H
+
+
+def _hook_times(vgv, kinds, run, reps=3):
+    """Per-kind launch durations (ms, minimum over reps) of one call of `run`,
+    from CUDA events the library records around each launch on its stream."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    evs = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in kinds}
+    for e0_, e1_ in evs.values():
+        e0_.record(stream)
+        e1_.record(stream)
+    torch.cuda.synchronize()
+    for k, (e0_, e1_) in evs.items():
+        vgv.vg_profile_set_events(k, [e0_], [e1_])
+    parts = {n: [] for n in kinds.values()}
+    try:
+        for _ in range(reps):
+            run()
+            torch.cuda.synchronize()
+            for k, (e0_, e1_) in evs.items():
+                parts[kinds[k]].append(e0_.elapsed_time(e1_))
+    finally:
+        for k in kinds:
+            vgv.vg_profile_set_events(k, [], [])
+    return {n: min(v) for n, v in parts.items()}
+
+
+def _event_ms(run, reps):
+    import torch
+
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        run()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_skewed(vgv, si, lm, dev, reps=10):
+    """The skewed-routing workload: one MoE layer over T = 4,096 tokens with the
+    per-expert logit bias 2 ln(1/(e+1)) (hot experts take most tokens, many take
+    none), then a K = 1 verify of 2,048 sequences x 2 rows of h = x + MoE(x) with
+    the full LM head. Reports the tensor fraction of both (CUDA events) and the
+    verified tokens/s."""
+    import torch
+
+    d = si.FULL
+    lw = si.torch_layer_weights(SEED, 4, 0, d, device=dev)
+    bias = torch.from_numpy(si.zipf_router_bias(E)).to(dev)
+    x = si.torch_normal_bf16((SKEW_T, H), 1.0, SEED, 4, si.TID_X, device=dev)
+    h = torch.empty_like(x)
+    ws = torch.empty(vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, SKEW_T), dtype=torch.uint8, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    taps = vgv.make_taps(expert_offsets=off)
+
+    def layer():
+        vgv.vg_moe_ffn(vgv.MOE_DIMS, SKEW_T, x, lw["router_w"], bias, lw["expert_w"], lw["shared_w"], 1, h, taps, ws)
+
+    layer_ms = _event_ms(layer, reps)
+    parts = _hook_times(vgv, {vgv.VG_KERNEL_ROUTER: "router", vgv.VG_KERNEL_GROUPING: "grouping",
+                              vgv.VG_KERNEL_EXPERTS: "expert_gemms", vgv.VG_KERNEL_COMBINE: "combine"}, layer)
+    cnt = (off[1:] - off[:-1]).cpu()
+    peak, kind = _bf16_peak()
+    gemm_flop = SKEW_FLOP - 2 * SKEW_T * E * H
+    R = SKEW_B * (SKEW_K + 1)
+    am = torch.empty(R, dtype=torch.int32, device=dev)
+    acc = torch.empty(SKEW_B, dtype=torch.int32, device=dev)
+    tok = torch.empty(SKEW_B, SKEW_K + 1, dtype=torch.int32, device=dev)
+    drafts = torch.zeros(SKEW_B, SKEW_K, dtype=torch.int32, device=dev)
+    wsv = torch.empty(vgv.vg_verify_workspace_bytes(SKEW_B, SKEW_K, H, V), dtype=torch.uint8, device=dev)
+
+    def verify():
+        vgv.vg_verify_greedy(SKEW_B, SKEW_K, H, V, h, lm, drafts, am, acc, tok, wsv)
+
+    verify()
+    torch.cuda.synchronize()
+    g = torch.Generator(device=dev)
+    g.manual_seed(SEED + 41)
+    a = am.view(SKEW_B, SKEW_K + 1)[:, :SKEW_K]
+    u = torch.rand(SKEW_B, SKEW_K, generator=g, device=dev)
+    noise = torch.randint(0, V, (SKEW_B, SKEW_K), generator=g, device=dev, dtype=torch.int32)
+    drafts.copy_(torch.where(u < P_DRAFT, a, noise))
+    ver_ms = _event_ms(verify, reps)
+    vparts = _hook_times(vgv, {vgv.VG_KERNEL_LM_HEAD: "lm_head", vgv.VG_KERNEL_ACCEPT: "accept"}, verify)
+    tokens = int((acc.to(torch.int64) + 1).sum().item())
+    del ws, wsv
+    return {"workload": f"one MoE layer, T={SKEW_T}, router bias 2 ln(1/(e+1)); then K=1 verify of "
+                        f"{SKEW_B} seqs x 2 rows with the full {V}-row LM head",
+            "expert_counts_max": int(cnt.max()), "experts_untouched": int((cnt == 0).sum()),
+            "layer_ms": layer_ms, "layer_tflops": SKEW_FLOP / (layer_ms / 1e3) / 1e12,
+            "expert_gemms_ms": parts["expert_gemms"],
+            "expert_gemms_tflops": gemm_flop / (parts["expert_gemms"] / 1e3) / 1e12,
+            "frac_layer": SKEW_FLOP / (layer_ms / 1e3) / 1e12 / peak,
+            "frac_expert_gemms": gemm_flop / (parts["expert_gemms"] / 1e3) / 1e12 / peak,
+            "breakdown_ms": parts,
+            "verify_ms": ver_ms, "verified_tokens": tokens, "verified_tokens_per_s": tokens / (ver_ms / 1e3),
+            "tau": tokens / SKEW_B, "lm_head_ms": vparts["lm_head"],
+            "lm_head_tflops": SKEW_LM_FLOP / (vparts["lm_head"] / 1e3) / 1e12,
+            "frac_lm_head": SKEW_LM_FLOP / (vparts["lm_head"] / 1e3) / 1e12 / peak,
+            "accept_ms": vparts["accept"],
+            "peak_tflops": peak, "peak_source": f"{kind} bf16_tflops (burst)"}
 
 
 def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
@@ -378,58 +513,107 @@ def _cores():
 
 # ------------------------------------------------------------------ oracle leg
 
-_ORACLE_INPUTS = {}
+def _oracle_threads():
+    """Threads the oracle's BLAS calls use (numpy's thread pool)."""
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return _cores()
 
 
-def oracle_step_sample(seed: int = SEED, n_sample: int = 2):
-    """Times the CPU oracle on a bounded sample of the step and scales it to a
-    whole step. Sample: n_sample of the 12 MoE layers over all 128 tokens (the
-    time of a layer is counted 12/n_sample times) plus the full LM-head argmax
-    and accept over the 128 rows. Inputs come from the numpy generator (same
-    distributions as the GPU leg) and are drawn once per process."""
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_step(layers, lm, x, drafts, Bq=B, Kq=K):
+    """One verify step of the CPU oracle, timed: the 12 MoE layers over the
+    B(K+1) rows, then the LM-head argmax and the prefix accept. Inputs are bf16
+    bits (uint16 arrays). Returns (seconds, verified tokens, argmax)."""
     import numpy as np
 
     import oracle
+
+    t0 = time.perf_counter()
+    h, _ = oracle.moe_stack(x, layers, k=TOPK, I=I)
+    arg, _ = oracle.lm_head_argmax(h, lm)
+    acc, _ = oracle.prefix_accept(arg, drafts, Bq, Kq)
+    return time.perf_counter() - t0, int(np.sum(acc + 1)), arg
+
+
+def oracle_one_thread(layers, lm, x, drafts):
+    """1-thread wall clock of the oracle on the tiny verify (1 layer, B=4, K=3,
+    16 rows) and on the batch-1 step (12 layers, B=1, K=3, 4 rows)."""
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=1):
+        s0, _, _ = oracle_step(layers[:1], lm, x[:16], drafts[:4], 4, K)
+        s2, _, _ = oracle_step(layers, lm, x[:4], drafts[:1], 1, K)
+    return {"tiny_verify_B4_K3_1_layer_s": s0, "batch1_K3_12_layers_s": s2}
+
+
+def _host_inputs(dev):
+    """The decode step's inputs as bf16 bits on the host: drawn by the seeded
+    torch generator (on the GPU when there is one, else on the CPU)."""
     import synth_inputs as si
 
     d = si.FULL
-    key = (seed, n_sample)
-    if key not in _ORACLE_INPUTS:
-        _ORACLE_INPUTS[key] = ([si.layer_weights(seed, CFG, l, d) for l in range(n_sample)],
-                               si.lm_head(seed, CFG, V, H), si.hidden_states(seed, CFG, T, H))
-    layers, lm, x = _ORACLE_INPUTS[key]
-    t0 = time.perf_counter()
-    h, _ = oracle.moe_stack(x, layers, k=TOPK, I=I)
-    t_layers = time.perf_counter() - t0
-    t1 = time.perf_counter()
-    arg, _ = oracle.lm_head_argmax(h, lm)
-    drafts = si.drafts_from_argmax(arg, B, K, P_DRAFT, V, seed, CFG)
-    acc, _ = oracle.prefix_accept(arg, drafts, B, K)
-    t_verify = time.perf_counter() - t1
-    step_s = t_layers * (LAYERS / n_sample) + t_verify
-    tokens = int(np.sum(acc + 1))
-    return step_s, tokens, (f"{n_sample} of {LAYERS} MoE layers over {T} tokens (time x{LAYERS / n_sample:g}) + "
-                            f"full LM-head argmax/accept over {T} rows")
+    layers = []
+    for l in range(LAYERS):
+        lw = si.torch_layer_weights(SEED, CFG, l, d, device=dev)
+        layers.append({k: si.torch_to_bits(v) for k, v in lw.items()})
+        del lw
+    lm = si.torch_to_bits(si.torch_normal_bf16((V, H), 0.02, SEED, CFG, si.TID_LM_HEAD, device=dev))
+    x = si.torch_to_bits(si.torch_normal_bf16((T, H), 1.0, SEED, CFG, si.TID_X, device=dev))
+    return layers, lm, x
 
 
 def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores: every step (warm-up and timed)
+    is one whole verify step of the workload, 12 layers + LM head + accept over
+    the 128 rows; the first warm-up step's argmax gives the drafts (p = 0.576)."""
     if rank != 0:
         return 0
-    for _ in range(args.warmup):
-        oracle_step_sample()
-    times, toks, sample = [], 0, ""
+    import numpy as np
+
+    import synth_inputs as si
+
+    try:
+        import torch
+
+        gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    except Exception:
+        gen_dev = "cpu"
+    layers, lm, x = _host_inputs(gen_dev)
+    drafts = np.zeros((B, K), dtype=np.int32)
+    for i in range(args.warmup):
+        _, _, arg = oracle_step(layers, lm, x, drafts)
+        if i == 0:
+            drafts = si.drafts_from_argmax(arg, B, K, P_DRAFT, V, SEED, CFG)
+    times, toks = [], 0
     for _ in range(args.steps):
-        s, toks, sample = oracle_step_sample()
-        times.append(s)
+        s_, toks, _ = oracle_step(layers, lm, x, drafts)
+        times.append(s_)
     step_s = statistics.mean(times)
     value = toks / step_s
-    cores = _cores()
+    sample = (f"one whole verify step per step: {LAYERS} MoE layers over {T} tokens + LM-head argmax/accept "
+              f"over {T} rows; numpy fp64 on {_cpu_model()}")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": dict(WORKLOAD, parallelism="host cores"),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -566,10 +750,11 @@ def run_gpu(args, rank, world, local):
         cur, nxt = nxt, cur
     del ws_one
     N = T * TOPK
-    # weights of every touched expert and the two shared ones; activations: token
-    # rows read, SwiGLU rows written and read back, expert outputs written
+    # algorithmic bytes of an expert-GEMM launch: the weights of every touched
+    # expert and the two shared ones, once; activations (token rows read, SwiGLU
+    # rows written and read back, expert outputs written) are reported apart
     act_bytes = N * H * 2 + T * H * 2 + 2 * (N + S * T) * I * 2 + (N + S * T) * H * 2
-    expert_bytes = [(n + S) * EXPERT_W_BYTES + act_bytes for n in n_touched]
+    expert_bytes = [(n + S) * EXPERT_W_BYTES for n in n_touched]
 
     # ---- device-timed region: the whole step replayed from a CUDA graph
     step(x, drafts)
@@ -671,6 +856,7 @@ def run_gpu(args, rank, world, local):
 
     # ---- the other shapes of the workload, measured on their own (untimed by the step)
     prefill = measure_prefill(vgv, si, dev) if not args.no_extra else None
+    skewed = measure_skewed(vgv, si, lm, dev) if not args.no_extra else None
     latency = measure_latency(vgv, x, rw, ew, sw, lm, dev) if not args.no_extra else None
     spec_loop = measure_spec_loop(vgv, si, rw, ew, sw, lm, dev) if not args.no_extra else None
     attention = measure_attention(vgv, si, dev) if not args.no_extra else None
@@ -680,10 +866,19 @@ def run_gpu(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s_step, s_tok, sample = oracle_step_sample()
-        cpu = {"value": s_tok / s_step, "unit": UNIT, "cores": _cores(), "kind": "oracle", "sample": sample}
+        # the oracle on the very same bytes: the step's inputs copied to the host
+        h_layers = [{k: si.torch_to_bits(v) for k, v in lw.items()} for lw in layers]
+        h_lm, h_x, h_d = si.torch_to_bits(lm), si.torch_to_bits(x), drafts.cpu().numpy()
+        s_step, s_tok, _ = oracle_step(h_layers, h_lm, h_x, h_d)
+        one = oracle_one_thread(h_layers, h_lm, h_x, h_d)
+        cpu = {"value": s_tok / s_step, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+               "sample": f"one whole verify step on the bench's inputs: {LAYERS} MoE layers over {T} tokens + "
+                         f"LM-head argmax/accept over {T} rows (numpy fp64)",
+               "step_s": s_step, "cpu_model": _cpu_model(), "one_thread_s": one}
+        del h_layers
 
     peak, peak_kind = _peaks()
+    step_bytes = step_weight_bytes(n_touched)
     line = {
         "metric": METRIC, "value": tokens_all / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -695,13 +890,25 @@ def run_gpu(args, rank, world, local):
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "kernel": "moe_expert_gemms (gate/up + SwiGLU + down, routed + shared)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": EXPERT_TRAFFIC_BYTES,
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": _traffic(EXPERT_TRAFFIC),
+                     "traffic_profile": EXPERT_TRAFFIC["profile"],
                      "algorithmic_bytes_per_launch": gu_bytes / max(1, len(gu)),
+                     "bytes_rule": "(touched routed experts + 2 shared) x 6,881,280 B of weights",
+                     "activation_bytes_per_launch": act_bytes,
+                     "n_touched_per_layer": n_touched,
                      "avg_launch_ms": sum(gu) / max(1, len(gu))},
+        "step_roofline": {"bound": "hbm", "algorithmic_bytes": step_bytes, "ms_per_step": ms,
+                          "achieved_gbs": step_bytes / (ms / 1e3) / 1e9,
+                          "frac_of_measured": step_bytes / (ms / 1e3) / 1e9 / peak,
+                          "frac_of_nominal_8tbs": step_bytes / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS,
+                          "measured_peak_gbs": peak, "peak_source": f"{peak_kind} hbm_gbs",
+                          "bytes_rule": "sum over layers of router + (touched + 2 shared) experts' weights, "
+                                        "+ the LM head; activations excluded"},
         "breakdown_ms_per_step": breakdown,
         "clocks": clk,
         "cpu_baseline": cpu,
         "prefill": prefill,
+        "skewed_routing": skewed,
         "batch1_latency": latency,
         "spec_decode_loop": spec_loop,
         "attention_layer": attention,

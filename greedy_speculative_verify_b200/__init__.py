@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "VG_OK", 1: "VG_ERR_INVALID_ARG", 2: "VG_ERR_UNSUPPORTED", 3:
 EXPORTS = (
     "vg_status_string", "vg_abi_version", "vg_moe_workspace_bytes", "vg_moe_ffn",
     "vg_moe_stack_workspace_bytes", "vg_moe_ffn_stack", "vg_verify_workspace_bytes",
-    "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag",
+    "vg_verify_greedy", "vg_get_device_status", "vg_set_wait_timeout_ns", "vg_debug_wait_flag", "vg_debug_wait_site",
     "vg_profile_set_events", "vg_profile_count", "vg_verify_greedy_noalloc",
     "vg_embed_rows", "vg_spec_rows", "vg_spec_commit", "vg_spec_rows_given",
     "vg_mtp_workspace_bytes", "vg_mtp_draft", "vg_attn_workspace_bytes", "vg_attn_verify",
@@ -97,6 +97,7 @@ def load():
         "vg_get_device_status": (i32, [vp, ctypes.POINTER(i32)]),
         "vg_set_wait_timeout_ns": (i32, [u64]),
         "vg_debug_wait_flag": (i32, [vp, i32, u64, vp]),
+        "vg_debug_wait_site": (i32, [i32, vp, u64, vp]),
         "vg_profile_set_events": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
         "vg_profile_count": (ctypes.c_int64, [i32]),
         "vg_verify_greedy_noalloc": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
@@ -206,6 +207,13 @@ def vg_set_wait_timeout_ns(ns: int):
 
 def vg_debug_wait_flag(flag, expect: int, max_ns: int, stream=None):
     _check(load().vg_debug_wait_flag(_ptr(flag), expect, max_ns, _stream(stream)), "vg_debug_wait_flag")
+
+
+VG_WAIT_MBARRIER, VG_WAIT_GRID_BARRIER = 1, 2
+
+
+def vg_debug_wait_site(which: int, ctr, max_ns: int, stream=None):
+    _check(load().vg_debug_wait_site(which, _ptr(ctr), max_ns, _stream(stream)), "vg_debug_wait_site")
 
 
 def vg_profile_set_events(kind: int, starts, stops):

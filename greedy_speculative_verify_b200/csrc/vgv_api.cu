@@ -645,6 +645,47 @@ extern "C" vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uin
   return cudaGetLastError() == cudaSuccess ? VG_OK : VG_ERR_CUDA;
 }
 
+namespace vg {
+// The pipeline-stage wait (mbar_wait) and the grid barrier, each made to run
+// out: no copy, MMA or other CTA's work is in flight when they give up.
+__global__ void debug_wait_site_kernel(int32_t which, uint32_t* ctr, uint64_t max_ns) {
+  if (which == VG_WAIT_MBARRIER) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+      mbar_init(&bar, 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, max_ns)) record_error(kErrTimeout, 903);
+  } else {
+    grid_barrier(ctr, gridDim.x + 1, max_ns, 902);  // one arrival more than the grid has CTAs
+  }
+}
+}  // namespace vg
+
+extern "C" vg_status vg_debug_wait_site(int32_t which, uint32_t* ctr, uint64_t max_ns, vg_stream_t stream) {
+  if ((which != VG_WAIT_MBARRIER && which != VG_WAIT_GRID_BARRIER) || max_ns == 0 || max_ns > 60000000000ull)
+    return VG_ERR_INVALID_ARG;
+  if (which == VG_WAIT_GRID_BARRIER && (ctr == nullptr || (reinterpret_cast<uintptr_t>(ctr) & 3u) != 0))
+    return VG_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (which == VG_WAIT_MBARRIER) {
+    vg::debug_wait_site_kernel<<<1, 32, 0, s>>>(which, ctr, max_ns);
+    return cudaGetLastError() == cudaSuccess ? VG_OK : cuda_fail();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, vg::debug_wait_site_kernel, which, ctr, max_ns) == cudaSuccess ? VG_OK
+                                                                                                : cuda_fail();
+}
+
 // ------------------------------------------------------------------ no-alloc
 // Scratch of vg_verify_greedy_noalloc: a file-scope device array (its host-side
 // name is only a stand-in; the device address comes from cudaGetSymbolAddress).
@@ -880,7 +921,7 @@ extern "C" vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w,
       !aligned16(hidden_out))
     return VG_ERR_INVALID_ARG;
   const MtpWs L = mtp_layout(B, w->V);
-  if (workspace == nullptr || workspace_bytes < L.total) return VG_ERR_WORKSPACE;
+  if (workspace == nullptr || workspace_bytes < L.total || !aligned16(workspace)) return VG_ERR_WORKSPACE;
   DevState* dev = nullptr;
   vg_status st = device_state(&dev);
   if (st != VG_OK) return st;
@@ -966,6 +1007,8 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   using namespace vg;
   if (B < 0 || K < 0 || K + 1 > kAttnMaxRows || L_max < 1 || L_max > 32768) return VG_ERR_INVALID_ARG;
   if (B == 0) return VG_OK;
+  // launch sizes count (row, head-pair) items in int
+  if ((int64_t)B * (K + 1) * kH >= ((int64_t)1 << 31)) return VG_ERR_UNSUPPORTED;
   if (!x || !w_qkv || !w_o || !kv_cache || !lens || !out) return VG_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(w_o) || !aligned16(kv_cache) || !aligned16(out) ||
       !aligned16(o_out))
@@ -977,7 +1020,7 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
                 overlaps(kv_cache, cache_bytes, o_out, rows_bytes)))
     return VG_ERR_INVALID_ARG;
   const AttnWs L = attn_layout(B, K, L_max);
-  if (workspace == nullptr || workspace_bytes < L.total) return VG_ERR_WORKSPACE;
+  if (workspace == nullptr || workspace_bytes < L.total || !aligned16(workspace)) return VG_ERR_WORKSPACE;
   DevState* dev = nullptr;
   vg_status st = device_state(&dev);
   if (st != VG_OK) return st;

@@ -49,7 +49,7 @@ typedef enum vg_status {
   VG_OK = 0,
   VG_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, aliasing, misalignment */
   VG_ERR_UNSUPPORTED = 2,   /* dimensions other than the supported shape */
-  VG_ERR_WORKSPACE = 3,     /* workspace null or smaller than the *_workspace_bytes query */
+  VG_ERR_WORKSPACE = 3,     /* workspace null, not 16-byte aligned, or smaller than the *_workspace_bytes query */
   VG_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
   VG_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (recorded in the status word) */
   VG_ERR_DEVICE_BOUNDS = 6  /* device: an index check failed (recorded in the status word) */
@@ -207,12 +207,27 @@ vg_status vg_get_device_status(vg_stream_t stream, int32_t* info);
  * the current device (default 4 s). Takes effect for launches after the call. */
 vg_status vg_set_wait_timeout_ns(uint64_t ns);
 
-/* Diagnostic: one thread waits (bounded by max_ns) until *flag == expect, using
- * the same bounded-wait code as the kernels' internal waits. A wait that runs
- * out records VG_ERR_TIMEOUT in the status word and returns; the context stays
- * usable. flag is an int32 device pointer. */
+/* Diagnostic: one thread polls (bounded by max_ns of %globaltimer) until
+ * *flag == expect. A wait that runs out records VG_ERR_TIMEOUT with site 901 in
+ * the status word and returns; the context stays usable. flag is an int32
+ * device pointer. */
 vg_status vg_debug_wait_flag(const int32_t* flag, int32_t expect, uint64_t max_ns,
                              vg_stream_t stream);
+
+/* Diagnostic of the two bounded waits inside the library's kernels, made to run
+ * out on purpose with no copy or tensor-core work in flight, through the same
+ * device functions the kernels call:
+ *   VG_WAIT_MBARRIER: one thread waits for a shared-memory mbarrier phase that
+ *     nothing completes (the wait of every TMA / MMA pipeline stage); site 903;
+ *   VG_WAIT_GRID_BARRIER: a cooperative launch of 2 CTAs waits at the grid
+ *     barrier of the layer-entry kernel for 3 arrivals, which never come;
+ *     ctr is a uint32 device word that must be 0 before the call; site 902.
+ * After max_ns (1 .. 60e9) the wait records VG_ERR_TIMEOUT with its site and
+ * the kernel returns; the context stays usable. Errors: VG_ERR_INVALID_ARG,
+ * VG_ERR_CUDA. */
+#define VG_WAIT_MBARRIER 1
+#define VG_WAIT_GRID_BARRIER 2
+vg_status vg_debug_wait_site(int32_t which, uint32_t* ctr, uint64_t max_ns, vg_stream_t stream);
 
 /* Allocation-free variant of vg_verify_greedy. The pages have no counterpart:
  * it exists for callers that cannot allocate device memory themselves — a
@@ -340,7 +355,8 @@ size_t vg_mtp_workspace_bytes(int32_t B, int32_t V);
  * states, K+1 and its accepted lengths). y0 int32 [B]. drafts int32 [B, K]
  * receives y_1 .. y_K; hidden_out, if not NULL, bf16 [K, B, H] receives
  * g_1 .. g_K. K = 0 or B = 0 is a no-op. Stream-ordered, capturable.
- * Errors: VG_ERR_INVALID_ARG, VG_ERR_WORKSPACE, VG_ERR_CUDA; a token outside
+ * Errors: VG_ERR_INVALID_ARG, VG_ERR_WORKSPACE (null, short or not 16-byte
+ * aligned), VG_ERR_CUDA; a token outside
  * [0, V) or an accepted length outside [0, rows_per_seq) records
  * VG_ERR_DEVICE_BOUNDS. */
 vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void* h, int32_t rows_per_seq,
@@ -371,7 +387,8 @@ vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void
  * probability-weighted sum of v) run on the tensor cores with bf16 operands and
  * fp32 accumulation, so the softmax weights enter the second product rounded to
  * bf16 (their sum is taken over the rounded weights). Errors: VG_ERR_INVALID_ARG,
- * VG_ERR_WORKSPACE, VG_ERR_CUDA.
+ * VG_ERR_UNSUPPORTED (B*(K+1)*H >= 2^31), VG_ERR_WORKSPACE (null, short or not
+ * 16-byte aligned), VG_ERR_CUDA.
  * ------------------------------------------------------------------------- */
 size_t vg_attn_workspace_bytes(int32_t B, int32_t K, int32_t L_max);
 vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const void* x, const void* w_qkv, const void* w_o,

@@ -154,6 +154,7 @@ def test_draft_block_validation_before_launch(lib):
     assert f(4, 3, ctypes.byref(w), None, 4, None, A, A, None, A, need, None) == 1    # h needed
     assert f(4, 3, ctypes.byref(w), A + 8, 4, None, A, A, None, A, need, None) == 1   # misaligned h
     assert f(4, 3, ctypes.byref(w), A, 4, None, A, A, None, A, need - 1, None) == 3   # short workspace
+    assert f(4, 3, ctypes.byref(w), A, 4, None, A, A, None, A + 8, need, None) == 3   # misaligned workspace
     bad = vgv.vg_mtp_weights(A, None, A, A, A, A, A, 1000)
     assert f(4, 3, ctypes.byref(bad), A, 4, None, A, A, None, A, need, None) == 1     # ffn needed
 
@@ -178,6 +179,8 @@ def test_attention_validation_before_launch(lib):
     assert f(*args(o=A + (3 << 30))) == 1         # o_out inside the cache
     assert f(*args(o=A + (7 << 30) + 8)) == 1     # misaligned o_out
     assert f(*args(n=need - 1)) == 3
+    assert f(*args(ws=A + (6 << 30) + 8)) == 3    # misaligned workspace
+    assert f(*args(B=600_000)) == 2               # B (K+1) H items overflow int launch sizes
 
 
 def test_attention_binding_checks_cache_shape():
@@ -191,3 +194,14 @@ def test_attention_binding_checks_cache_shape():
                 good.transpose(2, 3)):                                    # not dense
         with pytest.raises(ValueError):
             vgv.vg_attn_verify(2, 3, None, None, None, bad, None, None, None)
+
+
+def test_debug_wait_validation_before_launch(lib):
+    A = 1 << 40
+    f = lib.vg_debug_wait_site
+    assert f(0, A, 1000, None) == 1              # unknown wait kind
+    assert f(3, A, 1000, None) == 1
+    assert f(vgv.VG_WAIT_MBARRIER, A, 0, None) == 1           # zero limit
+    assert f(vgv.VG_WAIT_MBARRIER, A, 61_000_000_000, None) == 1  # over a minute
+    assert f(vgv.VG_WAIT_GRID_BARRIER, None, 1000, None) == 1     # the counter is needed
+    assert f(vgv.VG_WAIT_GRID_BARRIER, A + 2, 1000, None) == 1    # misaligned counter

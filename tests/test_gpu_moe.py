@@ -44,8 +44,9 @@ def _compare(g, r, T, check_act=True):
 def test_layer_parity(layer, T):
     """T=16: the tiny verify shape; 128: one decode layer at B=32, K=3; 2 and
     4: batch-1 K=1 / K=3; 200: several token tiles per shared expert with a
-    ragged tail; 1100 (> 512): the tiled router; 2000: 12,000 assignments take
-    the multi-kernel grouping path."""
+    ragged tail; 1100: 6,600 assignments, the layer-entry kernel with several
+    tokens per CTA (its largest sizes); 2000: 12,000 assignments take the
+    tiled router and the multi-kernel grouping path."""
     x = si.hidden_states(0, 1, T, D.H, tensor_id=100 + T)
     r = oracle.moe_ffn(x, layer["router_w"], layer["expert_w"], layer["shared_w"], k=D.k, I=D.I, add_residual=False)
     g = run_moe(x, layer, add_residual=False)

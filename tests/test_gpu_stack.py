@@ -7,7 +7,8 @@ import torch
 import greedy_speculative_verify_b200 as vgv
 import oracle
 import synth_inputs as si
-from gpu_common import ACT_TOL, D, assert_device_ok, dev, ensure_lib, f32, row_rel_err, run_moe, run_verify
+from gpu_common import (ACT_TOL, D, TIE_EPS, assert_device_ok, check_argmax, dev, ensure_lib, f32, row_rel_err,
+                        run_moe, run_verify)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,42 +64,73 @@ def test_stack_call_equals_layer_calls(stack):
     assert np.array_equal(si.torch_to_bits(cur), si.torch_to_bits(out))
 
 
-def test_chain_drift_then_verify(stack):
+def test_chain_stages_then_verify(stack, record_property):
     """x_{l+1} = bf16(x_l + MoE_l(x_l)) over the 12 layers, then verification.
 
-    The two chains round at different points: the GPU keeps the SwiGLU
-    activations and expert outputs in bf16 (2^-9 relative each), the oracle
-    keeps fp64 until the layer boundary. A bf16 boundary value then sometimes
-    rounds to the neighbouring number, and in later layers a token's 6th and 7th
-    experts can swap. An fp64 emulation of the GPU's rounding points on the same
-    shapes drifts from the oracle by 1.1% (median token) and 2.6% (worst token)
-    relative L2 after 12 layers; the bounds here are 2.5% and 6%.
-    Every argmax that differs on the final states must be explained by the
-    measured state difference: z_ref[a] - z_ref[g] <= ||h_gpu - h_ref|| *
-    ||LM_a - LM_g|| + the fp32 summation bound.
+    Greedy verification is lossless, so the result has an exact definition per
+    stage, but the two chains round at different points (the GPU keeps the
+    SwiGLU activations and expert outputs in bf16, the oracle fp64 until the
+    layer boundary), and after twelve layers their bf16 states differ. The
+    parity bar therefore applies per stage, on identical inputs:
+    * every layer along the GPU's own chain: routing ids and permutation
+      bit-exact against the oracle on the GPU's layer input, the layer's MoE
+      output within ACT_TOL, its residual output within ACT_TOL;
+    * the verify on the GPU's final states: argmax equal to the oracle's on the
+      same states (certified near-ties excepted), accepted lengths and
+      committed tokens equal to the prefix accept of that argmax.
+    Against the oracle's own fp64 chain the drift of the final states is only
+    reported (recorded as test properties), and each argmax that differs must be
+    explained by the measured state difference: with a the oracle-chain choice
+    and g the GPU's, z_ref[a] - z_ref[g] <= ||h_gpu - h_ref|| * ||LM_a - LM_g||
+    + the fp32 summation bound (Cauchy-Schwarz on the change of the logit
+    difference, which decides between a and g).
     """
     layers_dev, layers = stack
     x = si.hidden_states(0, 1, T, D.H)
-    ref_h, _ = oracle.moe_stack(x, layers, k=D.k, I=D.I)
+    cur = x
+    for l in range(L):
+        r = oracle.moe_ffn(cur, layers[l]["router_w"], layers[l]["expert_w"], layers[l]["shared_w"], k=D.k,
+                           I=D.I, add_residual=False)
+        g = run_moe(cur, layers_dev[l], add_residual=False)
+        assert np.array_equal(g["idx"], r["idx"]), l
+        assert np.array_equal(g["perm"], r["perm"]), l
+        assert row_rel_err(g["out"], r["out"]) <= ACT_TOL, l
+        g1 = run_moe(cur, layers_dev[l], add_residual=True)
+        assert np.array_equal(g1["idx"], r["idx"]), l
+        assert row_rel_err(g1["out"], f32(cur) + r["out"]) <= ACT_TOL, l
+        cur = si.f32_to_bf16_bits(g1["out"].astype(np.float32))
+    gpu_h = cur
     out = _run_stack(layers_dev, dev(x))
-    gpu_h = si.torch_to_bits(out)
-    rel = _row_rel_l2(f32(gpu_h), f32(ref_h))
-    assert np.median(rel) <= 0.025 and rel.max() <= 0.06, (np.median(rel), rel.max())
+    assert np.array_equal(si.torch_to_bits(out), gpu_h)  # the stack call takes the same chain
 
     lm_bits = si.lm_head(0, 1, D.V, D.H)
+    ref_h, _ = oracle.moe_stack(x, layers, k=D.k, I=D.I)
     ref_arg, _ = oracle.lm_head_argmax(ref_h, lm_bits)
     drafts = si.drafts_from_argmax(ref_arg, B, K, 0.576, D.V, seed=0, cfg=1)
     arg, acc, toks = run_verify(out, dev(lm_bits), drafts, B, K)
-    dh = f32(gpu_h) - f32(ref_h)
-    lmf = f32(lm_bits)
-    for r in np.nonzero(arg != ref_arg)[0]:
-        a, g = int(ref_arg[r]), int(arg[r])
-        z, amag = oracle.logit_fp64(ref_h, lm_bits, [r, r], [a, g])
-        bound = np.linalg.norm(dh[r]) * np.linalg.norm(lmf[a] - lmf[g]) + 2.0 ** -14 * amag.sum()
-        assert z[0] - z[1] <= bound, (r, a, g)
-    assert (arg == ref_arg).mean() >= 0.9
+    # verify stage on identical inputs (the GPU's final states)
+    own_arg, _ = oracle.lm_head_argmax(gpu_h, lm_bits)
+    check_argmax(arg, own_arg, gpu_h, lm_bits)
     a2, o2 = oracle.prefix_accept(arg, drafts, B, K)
     assert np.array_equal(acc, a2) and np.array_equal(toks, o2)
+
+    # chain level against the fp64 chain: reported, flips certified by the state difference
+    rel = _row_rel_l2(f32(gpu_h), f32(ref_h))
+    dh = f32(gpu_h) - f32(ref_h)
+    lmf = f32(lm_bits)
+    flips = np.nonzero(arg != ref_arg)[0]
+    for r in flips:
+        a, g = int(ref_arg[r]), int(arg[r])
+        z, amag = oracle.logit_fp64(ref_h, lm_bits, [r, r], [a, g])
+        bound = np.linalg.norm(dh[r]) * np.linalg.norm(lmf[a] - lmf[g]) + TIE_EPS * amag.sum()
+        assert z[0] - z[1] <= bound, (r, a, g)
+    ref_acc, _ = oracle.prefix_accept(ref_arg, drafts, B, K)
+    report = {"drift_rel_l2_median": float(np.median(rel)), "drift_rel_l2_max": float(rel.max()),
+              "argmax_flips_vs_fp64_chain": int(len(flips)),
+              "accepted_tokens_gpu": int((acc + 1).sum()), "accepted_tokens_fp64_chain": int((ref_acc + 1).sum())}
+    for k_, v_ in report.items():
+        record_property(k_, v_)
+    print("chain vs fp64 chain:", report)
 
 
 def test_bounded_wait_times_out_and_context_survives():
@@ -119,3 +151,25 @@ def test_bounded_wait_times_out_and_context_survives():
     g = run_moe(x, lw)
     r = oracle.moe_ffn(x, lw["router_w"], lw["expert_w"], lw["shared_w"], k=D.k, I=D.I)
     assert np.array_equal(g["idx"], r["idx"])
+
+
+@pytest.mark.parametrize("which,site", [(vgv.VG_WAIT_MBARRIER, 903), (vgv.VG_WAIT_GRID_BARRIER, 902)])
+def test_kernel_waits_time_out_and_context_survives(which, site):
+    """The pipeline-stage wait (an mbarrier phase nothing completes) and the
+    layer-entry grid barrier (one arrival short) run out after 2 ms through the
+    kernels' own wait functions, record VG_ERR_TIMEOUT with their site, and the
+    device keeps working."""
+    ensure_lib()
+    ctr = torch.zeros(1, dtype=torch.int32, device="cuda")
+    vgv.vg_debug_wait_site(which, ctr, 2_000_000)
+    st, info = vgv.vg_get_device_status()
+    assert st == 5 and info == site
+    assert vgv.vg_get_device_status() == (0, 0)
+    if which == vgv.VG_WAIT_GRID_BARRIER:
+        assert int(ctr.item()) == 2  # both CTAs arrived, the third arrival never came
+    lw = si.layer_weights(0, 12, 0, D)
+    x = si.hidden_states(0, 12, 8, D.H)
+    g = run_moe(x, lw)
+    r = oracle.moe_ffn(x, lw["router_w"], lw["expert_w"], lw["shared_w"], k=D.k, I=D.I)
+    assert np.array_equal(g["idx"], r["idx"])
+
