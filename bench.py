@@ -191,7 +191,7 @@ def _hook_times(vgv, kinds, run, reps=3):
     finally:
         for k in kinds:
             vgv.vg_profile_set_events(k, [], [])
-    return {n: min(v) for n, v in parts.items()}
+    return {n: (min(v) if v else None) for n, v in parts.items()}
 
 
 def _event_ms(run, reps):
@@ -241,7 +241,7 @@ def measure_skewed(vgv, si, lm, dev, reps=10):
     acc = torch.empty(SKEW_B, dtype=torch.int32, device=dev)
     tok = torch.empty(SKEW_B, SKEW_K + 1, dtype=torch.int32, device=dev)
     drafts = torch.zeros(SKEW_B, SKEW_K, dtype=torch.int32, device=dev)
-    wsv = torch.empty(vgv.vg_verify_workspace_bytes(SKEW_B, SKEW_K, H, V), dtype=torch.uint8, device=dev)
+    wsv = torch.zeros(vgv.vg_verify_workspace_bytes(SKEW_B, SKEW_K, H, V), dtype=torch.uint8, device=dev)
 
     def verify():
         vgv.vg_verify_greedy(SKEW_B, SKEW_K, H, V, h, lm, drafts, am, acc, tok, wsv)
@@ -255,7 +255,7 @@ def measure_skewed(vgv, si, lm, dev, reps=10):
     noise = torch.randint(0, V, (SKEW_B, SKEW_K), generator=g, device=dev, dtype=torch.int32)
     drafts.copy_(torch.where(u < P_DRAFT, a, noise))
     ver_ms = _event_ms(verify, reps)
-    vparts = _hook_times(vgv, {vgv.VG_KERNEL_LM_HEAD: "lm_head", vgv.VG_KERNEL_ACCEPT: "accept"}, verify)
+    vparts = _hook_times(vgv, {vgv.VG_KERNEL_LM_HEAD: "lm_head_argmax_accept"}, verify)
     tokens = int((acc.to(torch.int64) + 1).sum().item())
     del ws, wsv
     return {"workload": f"one MoE layer, T={SKEW_T}, router bias 2 ln(1/(e+1)); then K=1 verify of "
@@ -268,10 +268,9 @@ def measure_skewed(vgv, si, lm, dev, reps=10):
             "frac_expert_gemms": gemm_flop / (parts["expert_gemms"] / 1e3) / 1e12 / peak,
             "breakdown_ms": parts,
             "verify_ms": ver_ms, "verified_tokens": tokens, "verified_tokens_per_s": tokens / (ver_ms / 1e3),
-            "tau": tokens / SKEW_B, "lm_head_ms": vparts["lm_head"],
-            "lm_head_tflops": SKEW_LM_FLOP / (vparts["lm_head"] / 1e3) / 1e12,
-            "frac_lm_head": SKEW_LM_FLOP / (vparts["lm_head"] / 1e3) / 1e12 / peak,
-            "accept_ms": vparts["accept"],
+            "tau": tokens / SKEW_B, "lm_head_ms": vparts["lm_head_argmax_accept"],
+            "lm_head_tflops": SKEW_LM_FLOP / (vparts["lm_head_argmax_accept"] / 1e3) / 1e12,
+            "frac_lm_head": SKEW_LM_FLOP / (vparts["lm_head_argmax_accept"] / 1e3) / 1e12 / peak,
             "peak_tflops": peak, "peak_source": f"{kind} bf16_tflops (burst)"}
 
 
@@ -310,7 +309,7 @@ def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
         hid = torch.empty_like(x)
         am, acc, out = torch.empty(T_, **i32), torch.empty(B, **i32), torch.empty(B, K + 1, **i32)
         ws_s = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, T_), dtype=torch.uint8, device=dev)
-        ws_v = torch.empty(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
+        ws_v = torch.zeros(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
         st = vgv.make_spec_state(B, K, V, last, pos, committed, ref, p, SEED + 29, step, tokens, drafts if K else None)
 
         ws_m = torch.empty(vgv.vg_mtp_workspace_bytes(B, V), dtype=torch.uint8, device=dev) if mtp else None
@@ -387,7 +386,7 @@ def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
         ac = torch.empty(1, dtype=torch.int32, device=dev)
         tk = torch.empty(1, k + 1, dtype=torch.int32, device=dev)
         ws_s = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, t), dtype=torch.uint8, device=dev)
-        ws_v = torch.empty(vgv.vg_verify_workspace_bytes(1, k, H, V), dtype=torch.uint8, device=dev)
+        ws_v = torch.zeros(vgv.vg_verify_workspace_bytes(1, k, H, V), dtype=torch.uint8, device=dev)
 
         def step():
             vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, t, xk, rw, None, ew, sw, hid, ws_s)
@@ -723,7 +722,7 @@ def run_gpu(args, rank, world, local):
     accepted = torch.empty(B, dtype=torch.int32, device=dev)
     toks = torch.empty(B, K + 1, dtype=torch.int32, device=dev)
     ws_stack = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device=dev)
-    ws_ver = torch.empty(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
+    ws_ver = torch.zeros(vgv.vg_verify_workspace_bytes(B, K, H, V), dtype=torch.uint8, device=dev)
 
     def step(x_in, d_in):
         vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, T, x_in, rw, None, ew, sw, hid, ws_stack)
@@ -825,7 +824,7 @@ def run_gpu(args, rank, world, local):
     # is bracketed by event-record nodes; each replay is read before the next.
     kr = max(1, min(args.steps, 10))
     kinds = {vgv.VG_KERNEL_ROUTER: "layer_entry", vgv.VG_KERNEL_GROUPING: "grouping", vgv.VG_KERNEL_EXPERTS: "experts",
-             vgv.VG_KERNEL_COMBINE: "combine", vgv.VG_KERNEL_LM_HEAD: "lm_head", vgv.VG_KERNEL_ACCEPT: "accept"}
+             vgv.VG_KERNEL_COMBINE: "combine", vgv.VG_KERNEL_LM_HEAD: "lm_head_argmax_accept"}
     cap = LAYERS + 1  # no kind launches more often than this in one step
     evs = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(cap)],
                [torch.cuda.Event(enable_timing=True) for _ in range(cap)]) for k in kinds}

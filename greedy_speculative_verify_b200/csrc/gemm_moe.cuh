@@ -78,12 +78,20 @@ struct FusedArgs {
   int32_t* sched;          // [0]: ticket counter, [1 + t]: readiness of tile t; zero at launch
   __nv_bfloat16* act;      // [(k+S)T, I]: routed rows in permutation order, then shared
   __nv_bfloat16* out;      // [(k+S)T, H]: expert outputs, same rows
+  // 1: every expert has a primary tile (its first NMAX tokens, possibly none),
+  // tiles 0 .. E+S-1 in expert order, then the further tiles; CTA b's first unit
+  // is unit b (a gate/up unit of a primary tile, known before the routing), and
+  // its weights are requested before the kernel waits for the previous one
+  int32_t static_first;
+  int32_t pre_l2_chunks;   // static_first: k-chunks of the first unit past the stages, prefetched to L2
 };
 
 struct FgSched {
   int xrow[kMaxExperts];   // first row of the expert's tokens in its gate/up B map
   int arow[kMaxExperts];   // first row of the expert's activations / outputs
   int n[kMaxExperts];      // tokens of the expert
+  // first tile of each expert (static_first: first tile beyond its primary one,
+  // counted from tile E+S); pref[E+S] = the total
   int pref[kMaxExperts + 1];
 };
 
@@ -94,7 +102,8 @@ struct FgUnit {
 
 __device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, const FusedArgs& a, int nmax) {
   FgUnit un;
-  const int u1 = s.pref[n_exp] * a.mblk_gu;
+  const int n_tiles = s.pref[n_exp] + (a.static_first ? n_exp : 0);
+  const int u1 = n_tiles * a.mblk_gu;  // gate/up units come first
   int v = u, nm = a.mblk_gu;
   un.down = u >= u1;
   if (un.down) {
@@ -103,18 +112,25 @@ __device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, 
   }
   un.tile = v / nm;
   un.mb = v - un.tile * nm;
-  // the expert of the tile: the last e with pref[e] <= tile (experts without
-  // tokens have pref[e] == pref[e + 1] and are skipped by taking the last)
-  int lo = 0, hi = n_exp - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (s.pref[mid] <= un.tile) lo = mid;
-    else hi = mid - 1;
+  int e, nb;
+  if (a.static_first && un.tile < n_exp) {  // primary tile of expert `tile`
+    e = un.tile;
+    nb = 0;
+  } else {
+    // the expert of the tile: the last e with pref[e] <= t (experts without
+    // (further) tiles have pref[e] == pref[e + 1] and are skipped by taking the last)
+    const int t = a.static_first ? un.tile - n_exp : un.tile;
+    int lo = 0, hi = n_exp - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s.pref[mid] <= t) lo = mid;
+      else hi = mid - 1;
+    }
+    e = lo;
+    nb = t - s.pref[e] + (a.static_first ? 1 : 0);
   }
-  const int e = lo;
-  const int nb = un.tile - s.pref[e];
   un.e = e;
-  un.nrows = min(nmax, s.n[e] - nb * nmax);
+  un.nrows = max(0, min(nmax, s.n[e] - nb * nmax));  // 0 only for the primary tile of an expert without tokens
   un.xrow = s.xrow[e] + nb * nmax;
   un.arow = s.arow[e] + nb * nmax;
   return un;
@@ -173,6 +189,23 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // static_first: the weights of this CTA's first unit (gate/up of row block
+  // blockIdx.x % mblk_gu of expert blockIdx.x / mblk_gu) go out before the wait;
+  // its token rows follow once the routing is known
+  const int npre0 = args.static_first ? min(C::kStages, args.kc_gu) : 0;
+  if (npre0 > 0 && threadIdx.x == 0) {
+    const int e0 = blockIdx.x / args.mblk_gu, mb0 = blockIdx.x - e0 * args.mblk_gu;
+    const bool sh = e0 >= args.E;
+    const CUtensorMap* mA = sh ? &mGuS : &mGuR;
+    const int ec = sh ? e0 - args.E : e0;
+    const uint64_t pol_w = NMAX <= 64 ? policy_evict_first() : policy_evict_normal();
+    for (int kc = 0; kc < npre0; ++kc) {
+      mbar_expect_tx(&full[kc], C::kABytes);
+      tma_load_4d_hint(tiles + kc * C::kStageBytes, mA, &full[kc], kc * kBK, mb0 * kBM, 0, ec, pol_w);
+    }
+    const int kc1 = min(args.kc_gu, npre0 + args.pre_l2_chunks);
+    for (int kc = npre0; kc < kc1; ++kc) tma_prefetch_4d(mA, kc * kBK, mb0 * kBM, 0, ec);
+  }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&mGuR);
     prefetch_tmap(&mGuS);
@@ -207,7 +240,8 @@ __global__ void __launch_bounds__(192, 1)
       int acc = 0;
       for (int e = 0; e < n_exp; ++e) {
         sch->pref[e] = acc;
-        acc += cdiv(sch->n[e], NMAX);
+        const int nt = cdiv(sch->n[e], NMAX);
+        acc += args.static_first ? max(0, nt - 1) : nt;
       }
       sch->pref[n_exp] = acc;
     }
@@ -217,7 +251,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = *tmem_slot;
-  const int n_tiles = sch->pref[n_exp];
+  const int n_tiles = sch->pref[n_exp] + (args.static_first ? n_exp : 0);
   const int total = n_tiles * (args.mblk_gu + args.mblk_dn);
   const uint64_t limit = g_wait_timeout_ns;
   int32_t* ticket = args.sched;
@@ -241,11 +275,19 @@ __global__ void __launch_bounds__(192, 1)
         }
       };
       // the next ticket is requested one unit ahead so its round trip overlaps the loads
-      int next_u = atomicAdd(ticket, 1);
+      const int tbase = args.static_first ? (int)gridDim.x : 0;  // tickets after the fixed first units
+      int next_u = args.static_first ? (int)blockIdx.x : atomicAdd(ticket, 1);
+      bool pre_pending = npre0 > 0;  // stages 0 .. npre0-1 armed before the wait, not yet handed on
       while (true) {
         int u = next_u;
         if (u >= total || *abort_flag) u = -1;
-        if (u >= 0) next_u = atomicAdd(ticket, 1);
+        if (u >= 0) next_u = tbase + atomicAdd(ticket, 1);
+        const bool pre_unit = pre_pending && u >= 0;  // the first unit: its weight stages are armed
+        FgUnit un{};
+        if (u >= 0) {
+          un = fg_decode(u, *sch, n_exp, args, NMAX);
+          if (un.nrows == 0 && !pre_unit) continue;  // a tile without tokens: nothing to compute
+        }
         if (!mbar_wait(&uempty[slot], rphase ^ 1, limit)) {
           record_error(kErrTimeout, 130);
           *abort_flag = 1;
@@ -258,7 +300,16 @@ __global__ void __launch_bounds__(192, 1)
           rphase ^= 1;
         }
         if (u < 0) break;
-        const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
+        pre_pending = false;
+        if (un.nrows == 0) {
+          // the pre-armed unit of an expert no token chose: its weight copies
+          // complete the armed stages, which the MMA issuer then releases
+          for (int kc = 0; kc < npre0; ++kc) {
+            mbar_arrive(&full[stage]);
+            next_stage();
+          }
+          continue;
+        }
         const bool shared = un.e >= args.E;
         const int ecoord = shared ? un.e - args.E : un.e;
         const CUtensorMap* mA = un.down ? (shared ? &mDnS : &mDnR) : (shared ? &mGuS : &mGuR);
@@ -285,11 +336,15 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           uint8_t* st = tiles + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          if (un.down)
-            tma_load_3d_hint(st, mA, &full[stage], kc * kBK, arow, ecoord, pol_w);
-          else
-            tma_load_4d_hint(st, mA, &full[stage], kc * kBK, arow, 0, ecoord, pol_w);
+          if (pre_unit && kc < npre0) {  // weights in flight since before the wait
+            mbar_arrive_expect_tx(&full[stage], bytes - C::kABytes);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            if (un.down)
+              tma_load_3d_hint(st, mA, &full[stage], kc * kBK, arow, ecoord, pol_w);
+            else
+              tma_load_4d_hint(st, mA, &full[stage], kc * kBK, arow, 0, ecoord, pol_w);
+          }
           if (kc >= npre) load_b(stage, kc);
           if (kc + 1 == npre) {
             // every stage of the prefetch holds its weights in flight: now wait for the tile
@@ -308,6 +363,13 @@ __global__ void __launch_bounds__(192, 1)
           next_stage();
         }
         if (!ok) break;
+      }
+      if (pre_pending) {  // aborted before the first unit: complete its armed stages
+        for (int kc = 0; kc < npre0; ++kc) {
+          mbar_arrive(&full[kc]);
+          issued |= 1u << kc;
+          last_par &= ~(1u << kc);
+        }
       }
       // every issued copy has landed before the CTA may exit
       for (int s = 0; s < C::kStages; ++s)
@@ -332,6 +394,24 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (u < 0 || *abort_flag) break;
         const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
+        if (un.nrows == 0) {  // the pre-armed unit of an unused expert: release its stages
+          bool ok = true;
+          for (int kc = 0; kc < npre0; ++kc) {
+            if (!mbar_wait(&full[stage], phase, limit)) {
+              record_error(kErrTimeout, 138);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            mbar_arrive(&empty[stage]);
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (!ok) break;
+          continue;
+        }
         const int ab = lu & 1;
         const uint32_t ap = (lu >> 1) & 1;
         ++lu;
@@ -397,6 +477,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (u < 0 || *abort_flag) break;
       const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
+      if (un.nrows == 0) continue;  // nothing was computed for it
       const int ab = lu & 1;
       const uint32_t ap = (lu >> 1) & 1;
       ++lu;

@@ -61,6 +61,10 @@ struct EntryArgs {
   int32_t n_prefetch;
   uint32_t prefetch_bytes;
   uint64_t prefetch_stride;
+  // L2 prefetch by weight tile: the first pf_units gate/up units of the expert
+  // kernel's fixed first wave (unit u = row block u % mblk of routed expert
+  // u / mblk), pf_chunks 64-wide k-chunks each, through the gate/up tensor map
+  int32_t pf_units, pf_mblk, pf_chunks;
 };
 
 constexpr int kEntryH = 1280;                          // hidden size of the kernel
@@ -111,6 +115,7 @@ __device__ __forceinline__ void quarter_chains(const uint8_t* wq, int sw, const 
 
 template <int K>
 __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid_constant__ CUtensorMap mR,
+                                                                    const __grid_constant__ CUtensorMap mGu,
                                                                     const EntryArgs a) {
   constexpr int H = kEntryH, HQ = H / 4;
   extern __shared__ uint8_t esm_raw[];
@@ -144,7 +149,12 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
         tma_load_2d(ws + kc * 8192, &mR, &bars[0], kc * 64, 0);
       }
     }
-    if (a.n_prefetch > 0) {  // the first weights the expert kernel streams go to L2 now
+    // the first weights the expert kernel streams go to L2 now, while HBM is idle
+    for (int u = c; u < a.pf_units; u += G) {
+      const int e = u / a.pf_mblk, mb = u - e * a.pf_mblk;
+      for (int kc = 0; kc < a.pf_chunks; ++kc) tma_prefetch_4d(&mGu, kc * 64, mb * 128, 0, e);
+    }
+    if (a.n_prefetch > 0) {
       constexpr uint32_t kPiece = 1u << 20;
       const uint32_t pieces_per = cdiv((int)a.prefetch_bytes, (int)kPiece);
       for (uint32_t i = c; i < (uint32_t)a.n_prefetch * pieces_per; i += G) {

@@ -8,19 +8,18 @@
 // "Spekulatives Decoding auf einer L4"). Vocabulary 129,280 (jina-ocr-v1 model
 // card, architecture paragraph).
 //
-// lmhead_argmax: tcgen05 GEMM with the verify rows as M (128 per tile) and a
-// 176-row vocabulary slab as N; the fp32 logits never leave tensor memory. The
-// epilogue thread that owns row r scans its 176 columns in increasing vocabulary
-// order and keeps the best (value, index) as one 64-bit key: the order-
-// preserving image of the fp32 value in the high word and (2^32-1-v) in the low
-// word, so that the larger key is the larger logit and, among equal logits,
-// the lower index. A work unit is a group of consecutive vocabulary tiles for
-// one 128-row block; the key is carried across the group's tiles and one key
-// per (group, row) goes to the workspace.
-//
-// argmax_accept: reduces the keys of a row (max), writes argmax, and for each
-// sequence counts the leading drafts equal to the argmax of the preceding
-// position, then writes the committed tokens.
+// lmhead_argmax_accept: tcgen05 GEMM with the verify rows as M (128 per tile)
+// and a 176-row vocabulary slab as N; the fp32 logits never leave tensor
+// memory. The epilogue thread that owns row r scans its 176 columns in
+// increasing vocabulary order and keeps the best (value, index) as one 64-bit
+// key: the order-preserving image of the fp32 value in the high word and
+// (2^32-1-v) in the low word, so that the larger key is the larger logit and,
+// among equal logits, the lower index. A work unit is a group of consecutive
+// vocabulary tiles for one 128-row block; the key is carried across the
+// group's tiles and folded into the row's global key with an atomic max. The
+// last CTA to finish decodes the argmax, counts for each sequence the leading
+// drafts equal to the argmax of the preceding position, and writes the
+// committed tokens.
 #pragma once
 #include "common.cuh"
 
@@ -44,10 +43,28 @@ __device__ __forceinline__ uint64_t argmax_key(float z, uint32_t v) {
   return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - v);
 }
 
+struct LmArgs {
+  int R, V, k_chunks, n_mblk, n_vblk, group_tiles, n_groups, a_box_rows, b_box_rows;
+  int B, K;
+  const int32_t* drafts;         // [B, K]; may be null when K == 0
+  int32_t* argmax;               // [R]
+  int32_t* accepted;             // [B]
+  int32_t* out_tokens;           // [B, K+1]
+  unsigned long long* best;      // [R] running max key per row: zero at entry, left zero
+  uint32_t* done;                // CTAs finished: zero at entry, left zero
+};
+
+// Grid: one CTA per SM over units (vocabulary group, 128-row block). Before it
+// waits for the previous kernel, the producer already streams the vocabulary
+// tiles of its first stages (the LM head is immutable; only the hidden states
+// come from the previous kernel). Each unit folds its rows' best keys into
+// `best` with a 64-bit atomic max (order-independent, so the result does not
+// depend on the CTAs' timing); the last CTA to finish turns the keys into the
+// argmax, accepts each sequence's longest agreeing prefix plus the bonus token,
+// and clears `best` and `done` for the next call.
 __global__ void __launch_bounds__(192, 1)
-    lmhead_argmax(const __grid_constant__ CUtensorMap mapH, const __grid_constant__ CUtensorMap mapLM, int R,
-                  int V, int k_chunks, int n_mblk, int n_vblk, int group_tiles, int n_groups, int a_box_rows,
-                  int b_box_rows, uint64_t* __restrict__ part) {
+    lmhead_argmax_accept(const __grid_constant__ CUtensorMap mapH, const __grid_constant__ CUtensorMap mapLM,
+                         const LmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
@@ -59,8 +76,11 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ int last_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = a.n_groups * a.n_mblk;  // unit = (vocabulary group, row block), row block fastest
+  const uint32_t a_bytes = a.a_box_rows * kBK * 2, b_bytes = a.b_box_rows * kBK * 2;
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kLmStages; ++i) {
@@ -86,32 +106,44 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_wait();  // the hidden states come from the previous kernel
   const uint32_t tmem_base = *tmem_slot;
-  const int total = n_groups * n_mblk;  // unit = (vocabulary group, row block), row block fastest
   const uint64_t limit = g_wait_timeout_ns;
+
+  // vocabulary tiles of the first stages of this CTA's first unit, in the
+  // order the main loop consumes them: before the dependency wait
+  int npre = 0;
+  const uint64_t pol_w = policy_evict_first();
+  if (warp == 0 && lane == 0 && (int)blockIdx.x < total) {
+    const int g = blockIdx.x / a.n_mblk;
+    const int vb1 = min(a.n_vblk, (g + 1) * a.group_tiles);
+    for (int vb = g * a.group_tiles; vb < vb1 && npre < kLmStages; ++vb)
+      for (int kc = 0; kc < a.k_chunks && npre < kLmStages; ++kc, ++npre) {
+        mbar_expect_tx(&full[npre], b_bytes);
+        tma_load_2d_hint(tiles + npre * kLmStageBytes + kLmABytes, &mapLM, &full[npre], kc * kBK, vb * kLmN, pol_w);
+      }
+  }
+  griddep_wait();  // the hidden states (and the workspace) come from earlier kernels
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_h = policy_evict_last();
-      int stage = 0;
+      int stage = 0, it = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
-      const uint32_t bytes = (a_box_rows + b_box_rows) * kBK * 2;
       for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
-        const int g = u / n_mblk, mb = u - g * n_mblk;
-        const int vb1 = min(n_vblk, (g + 1) * group_tiles);
-        for (int vb = g * group_tiles; vb < vb1 && !*abort_flag; ++vb) {
-          for (int kc = 0; kc < k_chunks; ++kc) {
+        const int g = u / a.n_mblk, mb = u - g * a.n_mblk;
+        const int vb1 = min(a.n_vblk, (g + 1) * a.group_tiles);
+        for (int vb = g * a.group_tiles; vb < vb1 && !*abort_flag; ++vb) {
+          for (int kc = 0; kc < a.k_chunks; ++kc, ++it) {
             if (!mbar_wait(&empty[stage], phase ^ 1, limit)) {
               record_error(kErrTimeout, 121);
               *abort_flag = 1;
               break;
             }
             uint8_t* st = tiles + stage * kLmStageBytes;
-            mbar_arrive_expect_tx(&full[stage], bytes);
+            const bool pre = it < npre;  // its vocabulary tile is already in flight
+            mbar_arrive_expect_tx(&full[stage], pre ? a_bytes : a_bytes + b_bytes);
             tma_load_2d_hint(st, &mapH, &full[stage], kc * kBK, mb * kLmM, pol_h);
-            tma_load_2d_hint(st + kLmABytes, &mapLM, &full[stage], kc * kBK, vb * kLmN, pol_w);
+            if (!pre) tma_load_2d_hint(st + kLmABytes, &mapLM, &full[stage], kc * kBK, vb * kLmN, pol_w);
             issued |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);
             if (++stage == kLmStages) {
@@ -120,6 +152,13 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
+      }
+      // stages armed before the wait but never reached (an abort): arrive, so
+      // their copies complete the phase and can be drained below
+      for (; it < npre; ++it) {
+        mbar_arrive(&full[it]);
+        issued |= 1u << it;
+        last_par &= ~(1u << it);
       }
       for (int s = 0; s < kLmStages; ++s)
         if (issued & (1u << s)) mbar_wait(&full[s], (last_par >> s) & 1, limit);
@@ -132,9 +171,9 @@ __global__ void __launch_bounds__(192, 1)
       int lt = 0;  // local tile counter: selects the accumulator buffer
       bool ok = true;
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        const int g = u / n_mblk;
-        const int vb1 = min(n_vblk, (g + 1) * group_tiles);
-        for (int vb = g * group_tiles; vb < vb1 && ok; ++vb, ++lt) {
+        const int g = u / a.n_mblk;
+        const int vb1 = min(a.n_vblk, (g + 1) * a.group_tiles);
+        for (int vb = g * a.group_tiles; vb < vb1 && ok; ++vb, ++lt) {
           if (*abort_flag) {
             ok = false;
             break;
@@ -149,7 +188,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           tc_fence_after();
           const uint32_t d = tmem_base + ab * kLmAccCols;
-          for (int kc = 0; kc < k_chunks; ++kc) {
+          for (int kc = 0; kc < a.k_chunks; ++kc) {
             if (!mbar_wait(&full[stage], phase, limit)) {
               record_error(kErrTimeout, 123);
               *abort_flag = 1;
@@ -158,11 +197,11 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_fence_after();
             const uint32_t st = smem_u32(tiles + stage * kLmStageBytes);
-            const uint64_t a = sw128_kmajor_desc(st);
-            const uint64_t b = sw128_kmajor_desc(st + kLmABytes);
+            const uint64_t da = sw128_kmajor_desc(st);
+            const uint64_t db = sw128_kmajor_desc(st + kLmABytes);
 #pragma unroll
             for (int k16 = 0; k16 < kBK / 16; ++k16)
-              umma_bf16(d, a + 2 * k16, b + 2 * k16, idesc, (kc | k16) != 0);
+              umma_bf16(d, da + 2 * k16, db + 2 * k16, idesc, (kc | k16) != 0);
             umma_commit(&empty[stage]);
             if (++stage == kLmStages) {
               stage = 0;
@@ -181,10 +220,10 @@ __global__ void __launch_bounds__(192, 1)
     int lt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const int g = u / n_mblk, mb = u - g * n_mblk;
-      const int vb1 = min(n_vblk, (g + 1) * group_tiles);
+      const int g = u / a.n_mblk, mb = u - g * a.n_mblk;
+      const int vb1 = min(a.n_vblk, (g + 1) * a.group_tiles);
       uint64_t best = 0;  // running (value, index) key of this row over the group's tiles
-      for (int vb = g * group_tiles; vb < vb1; ++vb, ++lt) {
+      for (int vb = g * a.group_tiles; vb < vb1; ++vb, ++lt) {
         if (*abort_flag) {
           ok = false;
           break;
@@ -208,7 +247,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int v = v0 + c0 + j;
-            if (v < V) {
+            if (v < a.V) {
               const uint64_t key = argmax_key(__uint_as_float(z[j]), (uint32_t)v);
               best = key > best ? key : best;
             }
@@ -219,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(&tempty[ab]);
       }
       const int r = mb * kLmM + row;
-      if (ok && r < R) part[(size_t)g * R + r] = best;
+      if (ok && r < a.R) atomicMax(a.best + r, (unsigned long long)best);
     }
   }
   __syncthreads();
@@ -227,51 +266,32 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, kLmTmemCols);
   }
-}
 
-// One block handles whole sequences: spb = max(1, 32 / (K+1)) of them; its 32
-// warps reduce the rows' keys, then one thread per sequence accepts.
-__global__ void __launch_bounds__(1024) argmax_accept(const uint64_t* __restrict__ part, int n_groups, int R, int B,
-                                                      int K, const int32_t* __restrict__ drafts,
-                                                      int32_t* __restrict__ argmax, int32_t* __restrict__ accepted,
-                                                      int32_t* __restrict__ out_tokens) {
-  __shared__ int32_t arg_s[256];
-  griddep_launch_dependents();
-  griddep_wait();
-  const int spb = max(1, 32 / (K + 1));
-  const int seq0 = blockIdx.x * spb;
-  const int nseq = min(spb, B - seq0);
-  const int row0 = seq0 * (K + 1), nrows = nseq * (K + 1);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int rr = warp; rr < nrows; rr += 32) {
-    const int r = row0 + rr;
-    uint64_t best = 0;
-    for (int g = lane; g < n_groups; g += 32) {
-      const uint64_t k2 = part[(size_t)g * R + r];
-      best = k2 > best ? k2 : best;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = other > best ? other : best;
-    }
-    if (lane == 0) {
-      const int32_t a = (int32_t)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
-      arg_s[rr] = a;
-      argmax[r] = a;
-    }
+  // ---- the last CTA to finish: argmax, prefix accept, and the workspace back to zero
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's key updates precede its arrival
+    const uint32_t old = atomicAdd(a.done, 1u);
+    if (old >= gridDim.x) record_error(kErrBounds, 125);  // the counter was not zero at entry
+    last_s = old == gridDim.x - 1;
   }
   __syncthreads();
-  if ((int)threadIdx.x < nseq) {
-    const int b = seq0 + threadIdx.x;
-    const int32_t* arg = arg_s + threadIdx.x * (K + 1);
-    const int32_t* d = drafts + (size_t)b * K;
-    int a = 0;
-    while (a < K && d[a] == arg[a]) ++a;
-    accepted[b] = a;
-    int32_t* o = out_tokens + (size_t)b * (K + 1);
-    for (int i = 0; i <= K; ++i) o[i] = i < a ? d[i] : (i == a ? arg[a] : -1);
+  if (!last_s) return;
+  __threadfence();
+  for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+    const unsigned long long k = atomicExch(a.best + r, 0ull);
+    a.argmax[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
   }
+  __syncthreads();  // every argmax of this CTA is visible to all its threads
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+    const int32_t* arg = a.argmax + (size_t)b * (a.K + 1);
+    const int32_t* d = a.drafts + (size_t)b * a.K;
+    int acc = 0;
+    while (acc < a.K && d[acc] == arg[acc]) ++acc;
+    a.accepted[b] = acc;
+    int32_t* o = a.out_tokens + (size_t)b * (a.K + 1);
+    for (int i = 0; i <= a.K; ++i) o[i] = i < acc ? d[i] : (i == acc ? arg[acc] : -1);
+  }
+  if (threadIdx.x == 0) atomicExch(a.done, 0u);
 }
 
 }  // namespace vg

@@ -15,7 +15,9 @@
 #include "mtp.cuh"
 #include "attention.cuh"
 #include "gemm_moe.cuh"
+#include "gemm_tm.cuh"
 #include "layer_entry.cuh"
+#include "entry_small.cuh"
 #include "lmhead.cuh"
 #include "router.cuh"
 #include "sort.cuh"
@@ -25,6 +27,36 @@ namespace {
 constexpr int kH = 1280, kI = 896, kE = 64, kS = 2, kTopK = 6;
 constexpr int kMaxDevices = 64;
 constexpr int kEntryMaxGrid = 256;  // CTAs of the layer-entry kernel at most
+
+// Bytes of expert weights the layer entry prefetches into L2: the gate|up rows
+// of the first routed experts, which the expert kernel's first wave of units
+// streams (about one unit per SM).
+#ifndef VG_ENTRY_PREFETCH_MB
+#define VG_ENTRY_PREFETCH_MB 96
+#endif
+#ifndef VG_SMALL_ENTRY_PREFETCH_MB
+#define VG_SMALL_ENTRY_PREFETCH_MB 0
+#endif
+#ifndef VG_PRE_L2_CHUNKS
+#define VG_PRE_L2_CHUNKS 15
+#endif
+#ifndef VG_ENTRY_PF_UNITS
+#define VG_ENTRY_PF_UNITS 0
+#endif
+#ifndef VG_ENTRY_PF_CHUNKS
+#define VG_ENTRY_PF_CHUNKS 20
+#endif
+constexpr size_t kEntryPrefetchBytes = (size_t)VG_ENTRY_PREFETCH_MB << 20;
+// the two-token entry shares its SMs with the expert kernel, whose CTAs request
+// their first weights themselves; any prefetch of its own is on top of that
+constexpr size_t kSmallEntryPrefetchBytes = (size_t)VG_SMALL_ENTRY_PREFETCH_MB << 20;
+constexpr int kEntryPrefetchMinT = 64;  // 384 assignments: each expert untouched with probability < 0.3%
+// Static first units of the expert kernel (its first weights requested before
+// the routing is known) from this many tokens on, when the two-token entry runs:
+// then every expert is touched with probability > 99.7%, so the requested
+// weights are nearly always needed
+constexpr int kStaticFirstMinT = 64;
+constexpr int kPreL2Chunks = VG_PRE_L2_CHUNKS;  // further k-chunks of the first unit prefetched to L2
 
 struct DevState {
   bool init = false;
@@ -87,7 +119,9 @@ vg_status device_state(DevState** out) {
   DevState& d = g_dev[dev];
   if (!d.init) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cuda_fail();
-    if (cudaFuncSetAttribute(vg::moe_expert_gemms<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(vg::moe_expert_gemms_tm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::kTmSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vg::moe_expert_gemms<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::FgCfg<128>::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vg::moe_expert_gemms<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::FgCfg<64>::kSmemBytes) != cudaSuccess ||
@@ -100,9 +134,29 @@ vg_status device_state(DevState** out) {
     if (cudaFuncSetAttribute(vg::router_topk_tiled<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::kRtPartBytes) != cudaSuccess)
       return cuda_fail();
-    if (cudaFuncSetAttribute(vg::lmhead_argmax, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
+    if (cudaFuncSetAttribute(vg::lmhead_argmax_accept, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
       return cuda_fail();
+    // Kernels that follow each other with dependent launches share SMs only if
+    // their shared-memory configurations agree: every kernel of the decode
+    // chain asks for the largest shared-memory carveout.
+    {
+      const int kMax = cudaSharedmemCarveoutMaxShared;
+      const cudaFuncAttribute kC = cudaFuncAttributePreferredSharedMemoryCarveout;
+      if (cudaFuncSetAttribute(vg::moe_entry_small<kTopK>, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_layer_entry<kTopK>, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_expert_gemms<16>, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_expert_gemms<64>, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_expert_gemms<128>, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_expert_gemms_tm, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_combine, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::lmhead_argmax_accept, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::embed_rows, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::spec_rows, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::spec_rows_given, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::spec_commit, kC, kMax) != cudaSuccess)
+        return cuda_fail();
+    }
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -220,6 +274,24 @@ LayerBufs carve(void* workspace, int T, const vg_moe_taps* taps) {
   return b;
 }
 
+// Up to two tokens per CTA, next to the expert kernel (entry_small.cuh).
+bool entry_small_path(const DevState* dev, int T) {
+#ifndef VG_SMALL_ENTRY
+  (void)dev;
+  (void)T;
+  return false;  // measured slower than the one-token entry at 128 tokens: ~28 against ~18 us per layer
+#else
+  return vg::cdiv(T, vg::kEsTok) <= std::min(dev->sms, vg::kEsMaxGrid);
+#endif
+}
+bool static_first_units(const DevState* dev, int T) {
+#ifdef VG_NO_STATIC_FIRST
+  return false;
+#endif
+  return T >= kStaticFirstMinT && vg::cdiv(T, vg::kEsTok) <= std::min(dev->sms, vg::kEsMaxGrid) &&
+         expert_tile(T) == 64;
+}
+
 // The layer-entry kernel takes decode sizes: at most kEntryMaxOwn tokens per CTA
 // of its cooperative grid.
 int entry_grid(const DevState* dev, int T) {
@@ -242,8 +314,6 @@ struct PrevCombine {
 // Bytes of expert weights the layer entry prefetches into L2: the gate|up rows
 // of the first routed experts, which the expert kernel's first wave of units
 // streams (about one unit per SM).
-constexpr size_t kEntryPrefetchBytes = (size_t)96 << 20;
-constexpr int kEntryPrefetchMinT = 64;  // 384 assignments: each expert untouched with probability < 0.3%
 
 // Launch of a decode-path kernel with programmatic stream serialization (the
 // kernel waits for its predecessor itself, see griddep_wait), plain or
@@ -305,14 +375,36 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     a.n_prefetch = T >= kEntryPrefetchMinT ? (int)min((size_t)kE, kEntryPrefetchBytes / gu_bytes) : 0;
     a.prefetch_bytes = (uint32_t)gu_bytes;
     a.prefetch_stride = (uint64_t)3 * kI * kH * 2;
+    if (entry_small_path(dev, T)) {
+      const int grid = cdiv(T, kEsTok);
+      if (grid > 1) *nbar += 1;
+      a.n_prefetch = T >= kEntryPrefetchMinT ? (int)min((size_t)kE, kSmallEntryPrefetchBytes / gu_bytes) : 0;
+      ProfScope ps(VG_KERNEL_ROUTER, s);
+      if (launch_dep(moe_entry_small<kTopK>, grid, kEsThreads, 0, s, Launch::kCooperative,
+                     static_cast<const __nv_bfloat16*>(router_w), a) != cudaSuccess)
+        return cuda_fail();
+      return VG_OK;
+    }
     const int grid = entry_grid(dev, T);
     if (grid > 1) *nbar += 1;
-    CUtensorMap mR;
+    CUtensorMap mR, mGu;
     const uint64_t dR[2] = {kH, kE}, sR[1] = {kH * 2};
     const uint32_t bR[2] = {64, kE};
     if (make_map(&mR, router_w, 2, dR, sR, bR)) return VG_ERR_CUDA;
+    // tile prefetch of the expert kernel's first wave (its fixed first units)
+    // when those units are fixed; the map is the expert kernel's gate/up view
+    const uint64_t dGu[4] = {kH, kI, 2, kE};
+    const uint64_t sGu[3] = {kH * 2, (uint64_t)kI * kH * 2, (uint64_t)3 * kI * kH * 2};
+    const uint32_t bGu[4] = {kBK, kBM, 2, 1};
+    if (make_map(&mGu, expert_w, 4, dGu, sGu, bGu)) return VG_ERR_CUDA;
+    if (static_first_units(dev, T)) {
+      a.pf_mblk = kI / kBM;
+      a.pf_units = std::min(std::min(dev->sms, VG_ENTRY_PF_UNITS), kE * a.pf_mblk);
+      a.pf_chunks = VG_ENTRY_PF_CHUNKS;
+    }
     ProfScope ps(VG_KERNEL_ROUTER, s);
-    if (launch_dep(moe_layer_entry<kTopK>, grid, kEntryThreads, layer_entry_smem(), s, Launch::kCooperative, mR, a) != cudaSuccess)
+    if (launch_dep(moe_layer_entry<kTopK>, grid, kEntryThreads, layer_entry_smem(), s, Launch::kCooperative, mR, mGu,
+                   a) != cudaSuccess)
       return cuda_fail();
     return VG_OK;
   }
@@ -357,7 +449,15 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
   const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
   const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
-  const int nt = expert_tile(T), bx = std::min(kBoxRows, nt);  // a box never exceeds the token slot
+  const int nt = expert_tile(T);
+  // token-major kernel (128-token tiles): its token operand is one 128-row box;
+  // otherwise a box never exceeds the token slot
+#ifndef VG_PREFILL_WEIGHT_MAJOR
+  const bool tm = nt == 128;
+#else
+  const bool tm = false;
+#endif
+  const int bx = tm ? kTmM : std::min(kBoxRows, nt);
   const uint32_t bXr[2] = {kBK, (uint32_t)box_rows(N, bx)};
   const uint32_t bXs[2] = {kBK, (uint32_t)box_rows(T, bx)};
   const uint32_t bAct[2] = {kBK, (uint32_t)box_rows((int64_t)(kTopK + kS) * T, bx)};
@@ -382,9 +482,13 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   a.act = b.act;
   a.out = b.o;
   const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
+  a.static_first = static_first_units(dev, T) && grid <= (kE + kS) * a.mblk_gu ? 1 : 0;
+  a.pre_l2_chunks = kPreL2Chunks;
   ProfScope ps(VG_KERNEL_EXPERTS, s);
   const cudaError_t e =
-      nt == 16
+      tm ? launch_dep(moe_expert_gemms_tm, grid, 192, kTmSmemBytes, s, Launch::kPlain, mGuR, mGuS, mDnR, mDnS, mXr,
+                      mXs, mAct, a)
+      : nt == 16
           ? launch_dep(moe_expert_gemms<16>, grid, 192, FgCfg<16>::kSmemBytes, s, Launch::kPlain, mGuR, mGuS, mDnR, mDnS, mXr,
                        mXs, mAct, a)
       : nt == 64
@@ -419,10 +523,51 @@ vg_status launch_moe(DevState* dev, int T, const void* x, const void* router_w, 
   return st;
 }
 
+// Verify workspace: the running argmax key of every row, then the CTA counter.
 size_t verify_ws_bytes(int B, int K, int V) {
+  (void)V;
   const size_t R = (size_t)B * (K + 1);
-  const size_t ng = (size_t)vg::cdiv(vg::cdiv(V, vg::kLmN), vg::kLmGroupTiles);
-  return align256(ng * R * 8);
+  return align256(R * 8) + 256;
+}
+
+// The fused LM head + argmax + accept launch. `best` [R] and `done` must be
+// zero; the kernel leaves them zero.
+vg_status launch_verify(DevState* dev, int B, int K, int V, const void* h, const void* lm_head, const int32_t* drafts,
+                        int32_t* argmax, int32_t* accepted, int32_t* out_tokens, unsigned long long* best,
+                        uint32_t* done, cudaStream_t s) {
+  using namespace vg;
+  const int R = B * (K + 1);
+  LmArgs a{};
+  a.R = R;
+  a.V = V;
+  a.k_chunks = kH / kBK;
+  a.n_mblk = cdiv(R, kLmM);
+  a.n_vblk = cdiv(V, kLmN);
+  a.group_tiles = kLmGroupTiles;
+  a.n_groups = cdiv(a.n_vblk, kLmGroupTiles);
+  a.a_box_rows = box_rows(R, kLmM);
+  a.b_box_rows = box_rows(V, kLmN);
+  a.B = B;
+  a.K = K;
+  a.drafts = drafts;
+  a.argmax = argmax;
+  a.accepted = accepted;
+  a.out_tokens = out_tokens;
+  a.best = best;
+  a.done = done;
+  CUtensorMap mH, mLM;
+  {
+    const uint64_t dH[2] = {(uint64_t)kH, (uint64_t)R}, sH[1] = {(uint64_t)kH * 2};
+    const uint32_t bH[2] = {kBK, (uint32_t)a.a_box_rows};
+    const uint64_t dL[2] = {(uint64_t)kH, (uint64_t)V};
+    const uint32_t bL[2] = {kBK, (uint32_t)a.b_box_rows};
+    if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
+  }
+  const int grid = min(dev->sms, a.n_mblk * a.n_groups);
+  ProfScope ps(VG_KERNEL_LM_HEAD, s);
+  if (launch_dep(lmhead_argmax_accept, grid, 192, kLmSmemBytes, s, Launch::kPlain, mH, mLM, a) != cudaSuccess)
+    return cuda_fail();
+  return VG_OK;
 }
 
 }  // namespace
@@ -552,34 +697,10 @@ vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V, const voi
   DevState* dev = nullptr;
   vg_status st = device_state(&dev);
   if (st != VG_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int n_mblk = cdiv(R, kLmM), n_vblk = cdiv(V, kLmN);
-  const int a_box_rows = box_rows(R, kLmM);
-  CUtensorMap mH, mLM;
-  {
-    const uint64_t dH[2] = {(uint64_t)H, (uint64_t)R}, sH[1] = {(uint64_t)H * 2};
-    const uint32_t bH[2] = {kBK, (uint32_t)a_box_rows};
-    const uint64_t dL[2] = {(uint64_t)H, (uint64_t)V};
-    const uint32_t bL[2] = {kBK, (uint32_t)box_rows(V, kLmN)};
-    if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
-  }
-  uint64_t* part = static_cast<uint64_t*>(workspace);
-  const int n_groups = cdiv(n_vblk, kLmGroupTiles);
-  const int grid = min(dev->sms, n_mblk * n_groups);
-  {
-  ProfScope ps(VG_KERNEL_LM_HEAD, s);
-  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, Launch::kPlain, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
-                 kLmGroupTiles, n_groups, a_box_rows, box_rows(V, kLmN), part) != cudaSuccess)
-    return VG_ERR_CUDA;
-  }
-  const int spb = max(1, 32 / (K + 1));
-  {
-    ProfScope ps(VG_KERNEL_ACCEPT, s);
-    if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, Launch::kPlain, (const uint64_t*)part, n_groups, R, B, K, drafts,
-                   argmax, accepted, out_tokens) != cudaSuccess)
-      return VG_ERR_CUDA;
-  }
-  return VG_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return launch_verify(dev, B, K, V, h, lm_head, drafts, argmax, accepted, out_tokens,
+                       reinterpret_cast<unsigned long long*>(ws),
+                       reinterpret_cast<uint32_t*>(ws + align256((size_t)R * 8)), reinterpret_cast<cudaStream_t>(stream));
 }
 
 vg_status vg_get_device_status(vg_stream_t stream, int32_t* info) {
@@ -691,6 +812,7 @@ extern "C" vg_status vg_debug_wait_site(int32_t which, uint32_t* ctr, uint64_t m
 // name is only a stand-in; the device address comes from cudaGetSymbolAddress).
 namespace {
 constexpr size_t kNoAllocKeys = VG_NOALLOC_SCRATCH_BYTES / sizeof(uint64_t);
+constexpr size_t kNoAllocCounterSlots = 1;  // the last slot holds the CTA counter
 static __device__ __align__(256) uint64_t g_noalloc_scratch[kNoAllocKeys];
 uint64_t* g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
@@ -720,33 +842,17 @@ extern "C" vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, i
   if (!h || !lm_head || !argmax || !accepted || !out_tokens || (K > 0 && !drafts)) return VG_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(lm_head)) return VG_ERR_INVALID_ARG;
   const int R = B * (K + 1);
-  const int n_mblk = cdiv(R, kLmM), n_vblk = cdiv(V, kLmN);
-  const int n_groups = cdiv(n_vblk, kLmGroupTiles);
-  if ((uint64_t)n_groups * (uint64_t)R > kNoAllocKeys) return VG_ERR_WORKSPACE;
+  if ((uint64_t)R > kNoAllocKeys - kNoAllocCounterSlots) return VG_ERR_WORKSPACE;
   DevState* dev = nullptr;
   vg_status st = device_state(&dev);
   if (st != VG_OK) return st;
-  uint64_t* part = nullptr;
-  if ((st = noalloc_scratch(&part)) != VG_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int a_box_rows = box_rows(R, kLmM);
-  CUtensorMap mH, mLM;
-  {
-    const uint64_t dH[2] = {(uint64_t)H, (uint64_t)R}, sH[1] = {(uint64_t)H * 2};
-    const uint32_t bH[2] = {kBK, (uint32_t)a_box_rows};
-    const uint64_t dL[2] = {(uint64_t)H, (uint64_t)V};
-    const uint32_t bL[2] = {kBK, (uint32_t)box_rows(V, kLmN)};
-    if (make_map(&mH, h, 2, dH, sH, bH) || make_map(&mLM, lm_head, 2, dL, sH, bL)) return VG_ERR_CUDA;
-  }
-  const int grid = min(dev->sms, n_mblk * n_groups);
-  if (launch_dep(lmhead_argmax, grid, 192, kLmSmemBytes, s, Launch::kPlain, mH, mLM, R, V, H / kBK, n_mblk, n_vblk,
-                 kLmGroupTiles, n_groups, a_box_rows, box_rows(V, kLmN), part) != cudaSuccess)
-    return VG_ERR_CUDA;
-  const int spb = max(1, 32 / (K + 1));
-  if (launch_dep(argmax_accept, cdiv(B, spb), 1024, 0, s, Launch::kPlain, (const uint64_t*)part, n_groups, R, B, K, drafts,
-                 argmax, accepted, out_tokens) != cudaSuccess)
-    return VG_ERR_CUDA;
-  return VG_OK;
+  uint64_t* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != VG_OK) return st;
+  // keys in the first R slots, the CTA counter in the last slot: both zero at
+  // load time, and every call leaves them zero
+  return launch_verify(dev, B, K, V, h, lm_head, drafts, argmax, accepted, out_tokens,
+                       reinterpret_cast<unsigned long long*>(scratch),
+                       reinterpret_cast<uint32_t*>(scratch + kNoAllocKeys - 1), reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------ decode loop
@@ -929,7 +1035,11 @@ extern "C" vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(ws + o); };
   auto i32 = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
-  if (cudaMemsetAsync(ws + L.zero, 0, 16, s) != cudaSuccess) return cuda_fail();
+  // zero offsets of the dense products, and the verify workspace (the LM-head
+  // kernel needs it zero-filled and leaves it so)
+  if (cudaMemsetAsync(ws + L.zero, 0, 16, s) != cudaSuccess ||
+      cudaMemsetAsync(ws + L.vws, 0, verify_ws_bytes(B, 0, w->V), s) != cudaSuccess)
+    return cuda_fail();
   // g_i: in the caller's hidden_out when given, else in the workspace
   auto g_of = [&](int i) {
     return hidden_out ? static_cast<__nv_bfloat16*>(hidden_out) + (size_t)(i - 1) * B * kH : bf(L.g);

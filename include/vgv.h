@@ -142,7 +142,8 @@ vg_status vg_moe_ffn_stack(const vg_moe_dims* dims, int32_t n_layers, int32_t T,
                            void* out, void* workspace, size_t workspace_bytes,
                            vg_stream_t stream);
 
-/* Bytes of workspace vg_verify_greedy needs; 0 if the arguments are invalid. */
+/* Bytes of workspace vg_verify_greedy needs (8 per verify row + 256); 0 if the
+ * arguments are invalid. */
 size_t vg_verify_workspace_bytes(int32_t B, int32_t K, int32_t H, int32_t V);
 
 /* Greedy verification of B sequences with K drafted tokens each.
@@ -161,7 +162,16 @@ size_t vg_verify_workspace_bytes(int32_t B, int32_t K, int32_t H, int32_t V);
  *   argmax     int32 [B*(K+1)]   (out)
  *   accepted   int32 [B]         (out)
  *   out_tokens int32 [B, K+1]    (out)
- *   workspace  device buffer of at least vg_verify_workspace_bytes(B,K,H,V)
+ *   workspace  device buffer of at least vg_verify_workspace_bytes(B,K,H,V),
+ *              16-byte aligned, ZERO-FILLED before its first call (e.g.
+ *              cudaMemset to 0 once after allocating it); every call leaves it
+ *              zero-filled again, so it can be reused by later calls (one call
+ *              at a time) without clearing. It holds each row's running
+ *              argmax key and a counter of finished CTAs; a counter found
+ *              non-zero records VG_ERR_DEVICE_BOUNDS.
+ * One kernel launch: the LM-head GEMM, the argmax and the accept; the kernel
+ * starts streaming the LM head while the previous kernel in the stream is
+ * still running and reads h only after that kernel has finished.
  * H must be 1280; K >= 0; B*(K+1) < 2^24.
  * Errors: VG_ERR_INVALID_ARG, VG_ERR_UNSUPPORTED, VG_ERR_WORKSPACE, VG_ERR_CUDA. */
 vg_status vg_verify_greedy(int32_t B, int32_t K, int32_t H, int32_t V,
@@ -177,8 +187,9 @@ typedef enum vg_kernel {
   VG_KERNEL_EXPERTS = 2,   /* expert GEMMs: gate/up + SwiGLU, then down (one launch) */
   VG_KERNEL_COMBINE = 3,   /* weighted combine + shared experts + residual (a
                               layer's own output, or the stack's last layer) */
-  VG_KERNEL_LM_HEAD = 4,   /* LM-head GEMM + per-tile argmax */
-  VG_KERNEL_ACCEPT = 5,    /* argmax reduction + prefix accept */
+  VG_KERNEL_LM_HEAD = 4,   /* LM-head GEMM + argmax + prefix accept (one launch) */
+  VG_KERNEL_ACCEPT = 5,    /* kept for numbering: the accept now runs inside the
+                              LM-head launch, so nothing records this kind */
   VG_KERNEL_ATTENTION = 6, /* verifier attention: the chunk partials (scores,
                               softmax, values) of vg_attn_verify */
   VG_KERNEL_KINDS = 7
@@ -235,19 +246,19 @@ vg_status vg_debug_wait_site(int32_t which, uint32_t* ctr, uint64_t max_ns, vg_s
  * or a latency-critical loop that must not call cudaMalloc because it
  * synchronises the whole device — and so cannot provide a workspace.
  * Same computation, arguments and results as vg_verify_greedy, without the
- * workspace: the per-tile argmax keys go to a scratch array compiled into the
- * library (VG_NOALLOC_SCRATCH_BYTES = 2 MiB of device memory that every GPU
- * which loads the library holds until the process exits). Limit: one key per
- * (group of 5 vocabulary tiles of 176 rows, verify row),
- * ceil(ceil(V / 176) / 5) * B * (K+1) <= VG_NOALLOC_SCRATCH_BYTES / 8 = 262,144
- * keys (for V = 129,280: at most 1,783 verify rows); larger calls return
+ * workspace: the running argmax keys (8 bytes per verify row) and the kernel's
+ * counter of finished CTAs go to a scratch array compiled into the library
+ * (VG_NOALLOC_SCRATCH_BYTES = 2 MiB of device memory that every GPU which
+ * loads the library holds until the process exits). Limit: B * (K+1) <=
+ * VG_NOALLOC_SCRATCH_BYTES / 8 - 1 = 262,143 verify rows; larger calls return
  * VG_ERR_WORKSPACE and launch nothing. No call allocates or frees memory.
  * The first call on each device looks up the scratch array's device address
  * (with that device current) and caches it; make that first call before any
- * stream capture. Every call uses the same array: each call overwrites every
- * key it reads, so nothing needs clearing between calls, but calls whose work
- * overlaps on the GPU (different streams, or several threads) race on the
- * array and must be serialised by the caller. */
+ * stream capture. Every call uses the same array: it is zero when the library
+ * is loaded and every call leaves the part it used zero again, so nothing
+ * needs clearing between calls; but calls whose work overlaps on the GPU
+ * (different streams, or several threads) race on the array and must be
+ * serialised by the caller. */
 #define VG_NOALLOC_SCRATCH_BYTES (2u << 20)
 vg_status vg_verify_greedy_noalloc(int32_t B, int32_t K, int32_t H, int32_t V,
                                    const void* h, const void* lm_head, const int32_t* drafts,

@@ -44,6 +44,38 @@ def row_rel_err(gpu, ref):
     return float((np.abs(gpu - ref).max(axis=1) / den).max())
 
 
+GUARD_BYTES = 4096  # canary region on each side of every output buffer
+_CANARY = 0xA5
+
+
+class Guarded:
+    """Output tensors carved from the middle of larger buffers whose guard
+    regions (GUARD_BYTES on each side) hold a canary byte pattern; check()
+    asserts that no kernel wrote outside the tensors it was given. A stand-in
+    for a memory checker, which is not available on these GPUs."""
+
+    def __init__(self):
+        self.bufs = []
+
+    def empty(self, shape, dtype, fill=None):
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        raw = torch.full((nbytes + 2 * GUARD_BYTES,), _CANARY, dtype=torch.uint8, device="cuda")
+        t = raw[GUARD_BYTES:GUARD_BYTES + nbytes].view(dtype).view(*shape)
+        if fill is not None:
+            t.fill_(fill)
+        self.bufs.append((raw, nbytes))
+        return t
+
+    def check(self):
+        torch.cuda.synchronize()
+        for raw, nbytes in self.bufs:
+            head, tail = raw[:GUARD_BYTES], raw[GUARD_BYTES + nbytes:]
+            assert bool((head == _CANARY).all()) and bool((tail == _CANARY).all()), "write outside an output buffer"
+
+
 def assert_device_ok():
     st, info = vgv.vg_get_device_status()
     assert st == 0, f"device status {vgv.STATUS_NAMES.get(st, st)} at site {info}"
@@ -59,19 +91,21 @@ def run_moe(x_bits, lw, bias=None, add_residual=True, xdev=None):
     sw = lw["shared_w"] if torch.is_tensor(lw["shared_w"]) else dev(lw["shared_w"])
     b = None if bias is None else torch.from_numpy(np.asarray(bias, dtype=np.float32)).to(cuda)
     N = T * D.k
-    out = torch.empty(T, D.H, dtype=torch.bfloat16, device=cuda)
-    idx = torch.full((T, D.k), -1, dtype=torch.int32, device=cuda)
-    w = torch.empty(T, D.k, dtype=torch.float32, device=cuda)
-    off = torch.empty(D.E + 1, dtype=torch.int32, device=cuda)
-    perm = torch.empty(N, dtype=torch.int32, device=cuda)
-    inv = torch.empty(N, dtype=torch.int32, device=cuda)
-    act = torch.empty((D.k + D.S) * T, D.I, dtype=torch.bfloat16, device=cuda)
-    eo = torch.empty((D.k + D.S) * T, D.H, dtype=torch.bfloat16, device=cuda)
+    gd = Guarded()
+    out = gd.empty((T, D.H), torch.bfloat16)
+    idx = gd.empty((T, D.k), torch.int32, fill=-1)
+    w = gd.empty((T, D.k), torch.float32)
+    off = gd.empty((D.E + 1,), torch.int32)
+    perm = gd.empty((N,), torch.int32)
+    inv = gd.empty((N,), torch.int32)
+    act = gd.empty(((D.k + D.S) * T, D.I), torch.bfloat16)
+    eo = gd.empty(((D.k + D.S) * T, D.H), torch.bfloat16)
     taps = vgv.make_taps(idx, w, off, perm, inv, act, eo)
-    ws = torch.empty(vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device=cuda)
+    ws = gd.empty((vgv.vg_moe_workspace_bytes(vgv.MOE_DIMS, T),), torch.uint8)
     vgv.vg_moe_ffn(vgv.MOE_DIMS, T, x, rw, b, ew, sw, int(add_residual), out, taps, ws)
     torch.cuda.synchronize()
     assert_device_ok()
+    gd.check()
     return {
         "out": f32(si.torch_to_bits(out)), "idx": idx.cpu().numpy(), "g": w.cpu().numpy(),
         "offsets": off.cpu().numpy(), "perm": perm.cpu().numpy(), "inv": inv.cpu().numpy(),
@@ -88,13 +122,16 @@ def run_verify(h, lm, drafts, B, K, V=None):
     d = None
     if K > 0:
         d = drafts if torch.is_tensor(drafts) else torch.from_numpy(np.ascontiguousarray(drafts, dtype=np.int32)).to(cuda)
-    am = torch.full((max(R, 1),), -7, dtype=torch.int32, device=cuda)
-    acc = torch.full((max(B, 1),), -7, dtype=torch.int32, device=cuda)
-    ot = torch.full((max(B, 1), K + 1), -7, dtype=torch.int32, device=cuda)
-    ws = torch.empty(max(1, vgv.vg_verify_workspace_bytes(B, K, D.H, V)), dtype=torch.uint8, device=cuda)
+    gd = Guarded()
+    am = gd.empty((max(R, 1),), torch.int32, fill=-7)
+    acc = gd.empty((max(B, 1),), torch.int32, fill=-7)
+    ot = gd.empty((max(B, 1), K + 1), torch.int32, fill=-7)
+    ws = gd.empty((max(1, vgv.vg_verify_workspace_bytes(B, K, D.H, V)),), torch.uint8, fill=0)
     vgv.vg_verify_greedy(B, K, D.H, V, h, lm, d, am, acc, ot, ws)
     torch.cuda.synchronize()
     assert_device_ok()
+    gd.check()
+    assert int(ws.count_nonzero()) == 0  # the call leaves its workspace zero-filled
     return am.cpu().numpy(), acc.cpu().numpy(), ot.cpu().numpy()
 
 

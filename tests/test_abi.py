@@ -49,8 +49,9 @@ def test_workspace_queries(lib):
     assert vgv.vg_moe_stack_workspace_bytes(d, 128) >= w128 + 2 * 128 * 1280 * 2
     assert vgv.vg_moe_workspace_bytes(vgv.vg_moe_dims(1280, 896, 64, 2, 8), 128) == 0
     assert vgv.vg_moe_workspace_bytes(d, -1) == 0
-    groups = -(-(-(-129280 // 176)) // 5)  # 5 vocabulary tiles of 176 rows per key
-    assert vgv.vg_verify_workspace_bytes(32, 3, 1280, 129280) >= groups * 128 * 8
+    # one running argmax key per verify row, then the CTA counter
+    assert vgv.vg_verify_workspace_bytes(32, 3, 1280, 129280) == 128 * 8 + 256
+    assert vgv.vg_verify_workspace_bytes(1, 0, 1280, 129280) == 256 + 256
     assert vgv.vg_verify_workspace_bytes(32, 3, 1024, 129280) == 0
     assert vgv.vg_verify_workspace_bytes(32, -1, 1280, 129280) == 0
     assert vgv.vg_verify_workspace_bytes(1 << 22, 3, 1280, 129280) == 0

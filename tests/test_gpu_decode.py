@@ -45,7 +45,7 @@ class Decoder:
                                                                                          device="cuda")
         argmax, accepted, out = torch.empty(T, **i32), torch.empty(B, **i32), torch.empty(B, K + 1, **i32)
         ws_s = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, T), dtype=torch.uint8, device="cuda")
-        ws_v = torch.empty(vgv.vg_verify_workspace_bytes(B, K, D.H, V), dtype=torch.uint8, device="cuda")
+        ws_v = torch.zeros(vgv.vg_verify_workspace_bytes(B, K, D.H, V), dtype=torch.uint8, device="cuda")
         assert ref is None or ref.is_contiguous()  # read as [B, ref_len] rows
         st = vgv.make_spec_state(B, K, V, last, pos, committed, ref, p, seed, step, tokens, drafts if K else None)
         rw = [l["router_w"] for l in self.layers]

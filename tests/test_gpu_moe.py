@@ -40,13 +40,15 @@ def _compare(g, r, T, check_act=True):
     assert row_rel_err(g["out"], r["out"]) <= ACT_TOL
 
 
-@pytest.mark.parametrize("T", [1, 2, 4, 16, 128, 200, 1100, 2000])
+@pytest.mark.parametrize("T", [1, 2, 4, 16, 63, 64, 128, 200, 296, 297, 1100, 2000])
 def test_layer_parity(layer, T):
     """T=16: the tiny verify shape; 128: one decode layer at B=32, K=3; 2 and
-    4: batch-1 K=1 / K=3; 200: several token tiles per shared expert with a
-    ragged tail; 1100: 6,600 assignments, the layer-entry kernel with several
-    tokens per CTA (its largest sizes); 2000: 12,000 assignments take the
-    tiled router and the multi-kernel grouping path."""
+    4: batch-1 K=1 / K=3; up to 296 the two-token entry kernel (an odd T leaves
+    one CTA a single token; 296 fills 148 CTAs); from 64 on the expert kernel's
+    fixed first units (63 just below); 200: several token tiles per shared
+    expert with a ragged tail; 297 and 1100: the entry kernel with several
+    tokens per CTA; 2000: 12,000 assignments take the tiled router and the
+    multi-kernel grouping path."""
     x = si.hidden_states(0, 1, T, D.H, tensor_id=100 + T)
     r = oracle.moe_ffn(x, layer["router_w"], layer["expert_w"], layer["shared_w"], k=D.k, I=D.I, add_residual=False)
     g = run_moe(x, layer, add_residual=False)
@@ -65,6 +67,20 @@ def test_layer_skewed_routing(layer):
     r = oracle.moe_ffn(x, layer["router_w"], layer["expert_w"], layer["shared_w"], k=D.k, I=D.I, bias=bias,
                        add_residual=False)
     assert r["counts"][0] > 4000 and (r["counts"] == 0).sum() > 10
+    g = run_moe(x, layer, bias=bias, add_residual=False)
+    _compare(g, r, T)
+
+
+@pytest.mark.parametrize("T", [64, 128, 295])
+def test_decode_skewed_routing(layer, T):
+    """Decode sizes with the per-expert bias 2 ln(1/(e+1)): most experts get no
+    token, so the expert kernel's fixed first units of unused experts only
+    release their pipeline stages, and their further units are skipped."""
+    bias = si.zipf_router_bias(D.E)
+    x = si.hidden_states(0, 9, T, D.H, tensor_id=300 + T)
+    r = oracle.moe_ffn(x, layer["router_w"], layer["expert_w"], layer["shared_w"], k=D.k, I=D.I, bias=bias,
+                       add_residual=False)
+    assert (r["counts"] == 0).sum() > 20
     g = run_moe(x, layer, bias=bias, add_residual=False)
     _compare(g, r, T)
 

@@ -127,3 +127,45 @@ def test_verify_b_zero_writes_nothing(lm):
     vgv.vg_verify_greedy(0, 3, D.H, D.V, h, lm_t, am, am, am, am, None)
     torch.cuda.synchronize()
     assert torch.all(am == -7)
+
+
+def test_verify_leaves_workspace_zero_and_reports_a_dirty_counter(lm):
+    """The workspace (each row's running key, then the CTA counter) is left
+    zero-filled by every call. A counter that is not zero at entry is reported
+    as VG_ERR_DEVICE_BOUNDS (site 125) instead of being trusted; after clearing
+    it the next call is correct again."""
+    import greedy_speculative_verify_b200 as vgv
+
+    lm_bits, lm_t = lm
+    B, K = 8, 3
+    R = B * (K + 1)
+    h = si.hidden_states(0, 11, R, D.H, tensor_id=si.TID_HID)
+    ref_arg, _ = oracle.lm_head_argmax(h, lm_bits)
+    drafts = si.drafts_from_argmax(ref_arg, B, K, 0.576, D.V, seed=0, cfg=11)
+    cuda = torch.device("cuda")
+    ht, d = dev(h), torch.from_numpy(drafts).to(cuda)
+    am = torch.empty(R, dtype=torch.int32, device=cuda)
+    acc = torch.empty(B, dtype=torch.int32, device=cuda)
+    ot = torch.empty(B, K + 1, dtype=torch.int32, device=cuda)
+    nbytes = vgv.vg_verify_workspace_bytes(B, K, D.H, D.V)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=cuda)
+    for _ in range(2):
+        vgv.vg_verify_greedy(B, K, D.H, D.V, ht, lm_t, d, am, acc, ot, ws)
+        torch.cuda.synchronize()
+        assert vgv.vg_get_device_status() == (0, 0)
+        assert int(ws.count_nonzero()) == 0
+        check_argmax(am.cpu().numpy(), ref_arg, h, lm_bits)
+    counter = ws[(R * 8 + 255) // 256 * 256:].view(torch.int32)
+    counter[0] = 1000  # more than the grid has CTAs
+    vgv.vg_verify_greedy(B, K, D.H, D.V, ht, lm_t, d, am, acc, ot, ws)
+    torch.cuda.synchronize()
+    assert vgv.vg_get_device_status() == (6, 125)
+    ws.zero_()
+    am.fill_(-1)
+    vgv.vg_verify_greedy(B, K, D.H, D.V, ht, lm_t, d, am, acc, ot, ws)
+    torch.cuda.synchronize()
+    assert vgv.vg_get_device_status() == (0, 0)
+    check_argmax(am.cpu().numpy(), ref_arg, h, lm_bits)
+    a2, o2 = oracle.prefix_accept(am.cpu().numpy(), drafts, B, K)
+    assert np.array_equal(acc.cpu().numpy(), a2) and np.array_equal(ot.cpu().numpy(), o2)
+

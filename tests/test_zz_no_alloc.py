@@ -1,7 +1,8 @@
 """vg_verify_greedy_noalloc: the verify entry point for callers that cannot
 allocate device memory (a plugin whose memory belongs to its host
 application's pool, a loop that must not synchronise the device through
-cudaMalloc). It keeps its scratch in a fixed 2 MiB array inside the library
+cudaMalloc). It keeps its scratch (the running argmax key of each verify row
+and a counter of finished CTAs) in a fixed 2 MiB array inside the library
 instead of a caller-provided workspace.
 
 The GPU test calls it through the C ABI twice in a row, with different shapes,
@@ -40,7 +41,7 @@ def test_noalloc_matches_workspace_entry_two_calls():
         am0 = torch.empty(R, dtype=torch.int32, device=cuda)
         acc0 = torch.empty(B, dtype=torch.int32, device=cuda)
         tok0 = torch.empty(B, K + 1, dtype=torch.int32, device=cuda)
-        ws = torch.empty(vgv.vg_verify_workspace_bytes(B, K, D.H, D.V), dtype=torch.uint8, device=cuda)
+        ws = torch.zeros(vgv.vg_verify_workspace_bytes(B, K, D.H, D.V), dtype=torch.uint8, device=cuda)
         zeros = torch.zeros(B, K, dtype=torch.int32, device=cuda)
         vgv.vg_verify_greedy(B, K, D.H, D.V, h, lm, zeros, am0, acc0, tok0, ws)
         torch.cuda.synchronize()
@@ -61,13 +62,12 @@ def test_noalloc_matches_workspace_entry_two_calls():
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
-    """ceil(ceil(V/176)/5) * B*(K+1) keys must fit the 2 MiB array; a larger
-    call returns VG_ERR_WORKSPACE before any CUDA call (so this runs without a
-    GPU)."""
+    """One 8-byte key per verify row plus the counter slot must fit the 2 MiB
+    array (at most 262,143 rows); a larger call returns VG_ERR_WORKSPACE before
+    any CUDA call (so this runs without a GPU)."""
     lib = vgv.load()
     A = 1 << 40
-    groups = -(-(-(-D.V // 176)) // 5)
-    R_max = vgv.NOALLOC_SCRATCH_KEYS // groups
+    R_max = vgv.NOALLOC_SCRATCH_KEYS - 1
     B_bad = R_max // 4 + 1  # K = 3 -> 4 rows per sequence, just past the limit
     assert lib.vg_verify_greedy_noalloc(B_bad, 3, D.H, D.V, A, A, A, A, A, A, None) == 3
     assert lib.vg_verify_greedy_noalloc(0, 3, D.H, D.V, A, A, A, A, A, A, None) == 0
