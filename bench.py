@@ -372,11 +372,36 @@ def measure_spec_loop(vgv, si, rw, ew, sw, lm, dev, n_steps=20, p=P_DRAFT):
 
 def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
     """Batch-1 verify step latency (1 sequence, K = 3 and K = 1): 12 MoE layers,
-    LM-head argmax and accept, replayed from a CUDA graph."""
+    LM-head argmax and accept, replayed from a CUDA graph, two ways: the
+    multi-kernel path (layer stack + verify) and the single launch
+    (vg_verify_step_small). Bytes of a step: every layer's router, the experts
+    its rows touch (from the single launch's routing) and the two shared ones,
+    then the LM head."""
     import torch
 
     res = {}
     stream = torch.cuda.current_stream()
+    peak, _ = _peaks()
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        del g
+        return e0.elapsed_time(e1) / reps
+
+    ws_small = torch.empty(vgv.vg_verify_step_small_workspace_bytes(), dtype=torch.uint8, device=dev)
     for k in (3, 1):
         t = k + 1
         xk = x[:t].contiguous()
@@ -387,28 +412,33 @@ def measure_latency(vgv, x, rw, ew, sw, lm, dev, reps=20):
         tk = torch.empty(1, k + 1, dtype=torch.int32, device=dev)
         ws_s = torch.empty(vgv.vg_moe_stack_workspace_bytes(vgv.MOE_DIMS, t), dtype=torch.uint8, device=dev)
         ws_v = torch.zeros(vgv.vg_verify_workspace_bytes(1, k, H, V), dtype=torch.uint8, device=dev)
+        idx = torch.empty(LAYERS, t, TOPK, dtype=torch.int32, device=dev)
 
         def step():
             vgv.vg_moe_ffn_stack(vgv.MOE_DIMS, LAYERS, t, xk, rw, None, ew, sw, hid, ws_s)
             vgv.vg_verify_greedy(1, k, H, V, hid, lm, dr, am, ac, tk, ws_v)
 
-        step()
+        def one_launch(taps=False):
+            vgv.vg_verify_step_small(vgv.MOE_DIMS, LAYERS, 1, k, xk, rw, None, ew, sw, lm, V, dr, am, ac, tk,
+                                     ws_small, topk_idx_out=idx if taps else None)
+
+        res[f"K{k}_ms_per_step"] = timed(step)
+        one_launch(taps=True)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step()
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-        e1.synchronize()
-        res[f"K{k}_ms_per_step"] = e0.elapsed_time(e1) / reps
-        del g
-    res["workload"] = "B=1 verify step (K=3: 4 tokens, K=1: 2 tokens), 12 layers + LM head + accept, CUDA graph"
+        st, info = vgv.vg_get_device_status()
+        if st != 0:
+            raise RuntimeError(f"single-launch step: device status {st} at site {info}")
+        touched = [len(set(idx[l].flatten().tolist())) for l in range(LAYERS)]
+        nbytes = step_weight_bytes(touched)
+        ms1 = timed(one_launch)
+        res[f"K{k}_one_launch"] = {"ms_per_step": ms1, "algorithmic_bytes": nbytes,
+                                   "touched_experts_per_layer": touched,
+                                   "achieved_gbs": nbytes / (ms1 / 1e3) / 1e9,
+                                   "frac_of_measured_hbm": nbytes / (ms1 / 1e3) / 1e9 / peak,
+                                   "frac_of_nominal_8tbs": nbytes / (ms1 / 1e3) / 1e9 / NOMINAL_HBM_GBS}
+        res[f"K{k}_multi_kernel_frac_of_measured_hbm"] = nbytes / (res[f"K{k}_ms_per_step"] / 1e3) / 1e9 / peak
+    res["workload"] = ("B=1 verify step (K=3: 4 tokens, K=1: 2 tokens), 12 layers + LM head + accept, CUDA graph; "
+                       "multi-kernel path and single launch")
     return res
 
 

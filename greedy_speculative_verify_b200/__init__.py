@@ -30,6 +30,7 @@ EXPORTS = (
     "vg_profile_set_events", "vg_profile_count", "vg_verify_greedy_noalloc",
     "vg_embed_rows", "vg_spec_rows", "vg_spec_commit", "vg_spec_rows_given",
     "vg_mtp_workspace_bytes", "vg_mtp_draft", "vg_attn_workspace_bytes", "vg_attn_verify",
+    "vg_verify_step_small_workspace_bytes", "vg_verify_step_small",
 )
 
 # vg_kernel
@@ -109,6 +110,10 @@ def load():
         "vg_mtp_draft": (i32, [i32, i32, ctypes.POINTER(vg_mtp_weights), vp, i32, vp, vp, vp, vp, vp, sz, vp]),
         "vg_attn_workspace_bytes": (sz, [i32, i32, i32]),
         "vg_attn_verify": (i32, [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "vg_verify_step_small_workspace_bytes": (sz, []),
+        "vg_verify_step_small": (i32, [dims_p, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                       ctypes.POINTER(vp), ctypes.POINTER(vp), vp, i32, vp, vp, vp, vp, vp, vp,
+                                       vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -192,6 +197,27 @@ def vg_verify_greedy(B, K, H, V, h, lm_head, drafts, argmax, accepted, out_token
                                  0 if workspace is None else workspace.numel() * workspace.element_size(),
                                  _stream(stream))
     _check(st, "vg_verify_greedy")
+
+
+def vg_verify_step_small_workspace_bytes() -> int:
+    return load().vg_verify_step_small_workspace_bytes()
+
+
+def vg_verify_step_small(dims, n_layers, B, K, x, router_w, router_bias, expert_w, shared_w, lm_head, V, drafts,
+                         argmax, accepted, out_tokens, workspace, states_out=None, topk_idx_out=None, stream=None):
+    """The whole verify step (n_layers MoE layers, LM-head argmax, accept) for
+    B (K+1) <= 16 rows in one launch. Sequences of n_layers tensors as in
+    vg_moe_ffn_stack."""
+    arr = ctypes.c_void_p * n_layers
+    rw = arr(*(t.data_ptr() for t in router_w))
+    ew = arr(*(t.data_ptr() for t in expert_w))
+    sw = arr(*(t.data_ptr() for t in shared_w))
+    rb = None if router_bias is None else arr(*(None if t is None else t.data_ptr() for t in router_bias))
+    st = load().vg_verify_step_small(ctypes.byref(dims), n_layers, B, K, _ptr(x), rw, rb, ew, sw, _ptr(lm_head), V,
+                                     _ptr(drafts), _ptr(argmax), _ptr(accepted), _ptr(out_tokens),
+                                     _ptr(states_out), _ptr(topk_idx_out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "vg_verify_step_small")
 
 
 def vg_get_device_status(stream=None) -> tuple[int, int]:

@@ -73,6 +73,7 @@ constexpr int kEntryGroupTok = 2;                      // tokens per group and p
 constexpr int kEntryPassTok = 2 * kEntryGroupTok;      // tokens per pass
 constexpr int kEntryMaxOwn = 12;                       // tokens a CTA may own (T <= 12 * grid)
 constexpr int kEntrySlices = kEntryThreads / kRouterE; // CTA slices in the offsets phase
+constexpr int kEntryMaxGridDev = 160;                  // CTAs of the kernel at most (the host keeps grid <= SMs <= this)
 
 // Shared memory: router tiles, owned token rows (bf16), the pass's rows in
 // fp32, plus 1 KB alignment slack.
@@ -272,11 +273,17 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
     int* red = reinterpret_cast<int*>(&part[0][0][0]);  // [2][kEntrySlices][64]
     const int s = tid >> 6;
     int tot = 0, pre = 0;
-#pragma unroll 4
-    for (int cc = s; cc < G; cc += kEntrySlices) {
-      const int v = __ldcg(a.counts + (size_t)cc * kRouterE + e);
-      tot += v;
-      pre += cc < c ? v : 0;
+    // every count this thread needs is requested at once: one L2 round trip
+    int v[kEntryMaxGridDev / kEntrySlices];
+#pragma unroll
+    for (int i = 0; i < kEntryMaxGridDev / kEntrySlices; ++i) {
+      const int cc = s + i * kEntrySlices;
+      v[i] = cc < G ? __ldcg(a.counts + (size_t)cc * kRouterE + e) : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < kEntryMaxGridDev / kEntrySlices; ++i) {
+      tot += v[i];
+      pre += s + i * kEntrySlices < c ? v[i] : 0;
     }
     red[s * kRouterE + e] = tot;
     red[(kEntrySlices + s) * kRouterE + e] = pre;

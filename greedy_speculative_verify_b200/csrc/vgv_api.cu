@@ -20,6 +20,7 @@
 #include "entry_small.cuh"
 #include "lmhead.cuh"
 #include "router.cuh"
+#include "step_small.cuh"
 #include "sort.cuh"
 
 namespace {
@@ -133,6 +134,9 @@ vg_status device_state(DevState** out) {
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::router_topk_tiled<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::kRtPartBytes) != cudaSuccess)
+      return cuda_fail();
+    if (cudaFuncSetAttribute(vg::verify_step_small<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vg::kSsSmemBytes) != cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax_accept, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
@@ -295,7 +299,7 @@ bool static_first_units(const DevState* dev, int T) {
 // The layer-entry kernel takes decode sizes: at most kEntryMaxOwn tokens per CTA
 // of its cooperative grid.
 int entry_grid(const DevState* dev, int T) {
-  return std::min(std::min(dev->sms, kEntryMaxGrid), T);
+  return std::min(std::min(std::min(dev->sms, kEntryMaxGrid), vg::kEntryMaxGridDev), T);
 }
 bool small_path(const DevState* dev, int T) {
   return (int64_t)T * kTopK <= vg::kSortSmallMax && vg::cdiv(T, entry_grid(dev, T)) <= vg::kEntryMaxOwn;
@@ -1188,5 +1192,119 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   if (launch_dep(attn_residual, cdiv(R * kH / 4, 256), 256, 0, s, Launch::kPlain, static_cast<const __nv_bfloat16*>(x),
                  (const float*)pk, kProjSplits, R * kH, static_cast<__nv_bfloat16*>(out)) != cudaSuccess)
     return cuda_fail();
+  return VG_OK;
+}
+
+// ------------------------------------------------------------ small-batch step
+namespace {
+struct SsWs {
+  size_t ctrl, part_gu, part_dn, act, o, total;
+};
+SsWs ss_layout() {
+  using namespace vg;
+  SsWs L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.ctrl = take(sizeof(SsCtrl));
+  L.part_gu = take((size_t)kSsSlots * kSsMbGu * kSsKsGu * kSsPartFloats * 4);
+  L.part_dn = take((size_t)kSsSlots * kSsMbDn * kSsKsDn * kSsPartFloats * 4);
+  L.act = take((size_t)kSsSlots * kSsN * kI * 2);
+  L.o = take((size_t)kSsSlots * kSsN * kH * 2);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+extern "C" size_t vg_verify_step_small_workspace_bytes(void) { return ss_layout().total; }
+
+extern "C" vg_status vg_verify_step_small(const vg_moe_dims* dims, int32_t n_layers, int32_t B, int32_t K,
+                                          const void* x, const void* const* router_w,
+                                          const float* const* router_bias, const void* const* expert_w,
+                                          const void* const* shared_w, const void* lm_head, int32_t V,
+                                          const int32_t* drafts, int32_t* argmax, int32_t* accepted,
+                                          int32_t* out_tokens, void* states_out, int32_t* topk_idx_out,
+                                          void* workspace, size_t workspace_bytes, vg_stream_t stream) {
+  using namespace vg;
+  if (dims == nullptr || B < 0 || K < 0 || V < 1 || n_layers < 1 || !router_w || !expert_w || !shared_w)
+    return VG_ERR_INVALID_ARG;
+  if (!dims_supported(dims) || n_layers > kSsMaxLayers || (int64_t)B * (K + 1) > kSsN) return VG_ERR_UNSUPPORTED;
+  if (B == 0) return VG_OK;
+  if (!x || !lm_head || !argmax || !accepted || !out_tokens || (K > 0 && !drafts)) return VG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(lm_head) || !aligned16(states_out)) return VG_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (!router_w[l] || !expert_w[l] || !shared_w[l] || !aligned16(router_w[l]) || !aligned16(expert_w[l]) ||
+        !aligned16(shared_w[l]))
+      return VG_ERR_INVALID_ARG;
+  const SsWs W = ss_layout();
+  if (workspace == nullptr || workspace_bytes < W.total || !aligned16(workspace)) return VG_ERR_WORKSPACE;
+  DevState* dev = nullptr;
+  vg_status st = device_state(&dev);
+  if (st != VG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  SsMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const uint64_t estride = (uint64_t)3 * kI * kH * 2;
+  const uint64_t dGu[4] = {kH, kI, 2, kE}, dGuS[4] = {kH, kI, 2, kS};
+  const uint64_t sGu[3] = {kH * 2, (uint64_t)kI * kH * 2, estride};
+  const uint32_t bGu[4] = {kBK, kBM, 2, 1};
+  const uint64_t dDn[3] = {kI, kH, kE}, dDnS[3] = {kI, kH, kS}, sDn[2] = {kI * 2, estride};
+  const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
+  for (int l = 0; l < n_layers; ++l) {
+    const __nv_bfloat16* dr = static_cast<const __nv_bfloat16*>(expert_w[l]) + (size_t)2 * kI * kH;
+    const __nv_bfloat16* dsh = static_cast<const __nv_bfloat16*>(shared_w[l]) + (size_t)2 * kI * kH;
+    if (make_map(&maps.gu[l][0], expert_w[l], 4, dGu, sGu, bGu) ||
+        make_map(&maps.gu[l][1], shared_w[l], 4, dGuS, sGu, bGu) || make_map(&maps.dn[l][0], dr, 3, dDn, sDn, bDn) ||
+        make_map(&maps.dn[l][1], dsh, 3, dDnS, sDn, bDn))
+      return VG_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  {
+    const uint64_t dA[2] = {kI, (uint64_t)kSsSlots * kSsN}, sA[1] = {kI * 2};
+    const uint32_t bA[2] = {kBK, kSsN};
+    const uint64_t dL[2] = {kH, (uint64_t)V}, sL[1] = {kH * 2};
+    const uint32_t bL[2] = {kBK, (uint32_t)box_rows(V, kBM)};
+    if (make_map(&maps.act, ws + W.act, 2, dA, sA, bA) || make_map(&maps.lm, lm_head, 2, dL, sL, bL))
+      return VG_ERR_CUDA;
+  }
+  if (V < kBM) return VG_ERR_UNSUPPORTED;  // the LM-head units read 128-row boxes
+  SsArgs a{};
+  a.T = B * (K + 1);
+  a.B = B;
+  a.K = K;
+  a.L = n_layers;
+  a.V = V;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  for (int l = 0; l < n_layers; ++l) {
+    a.router_w[l] = static_cast<const __nv_bfloat16*>(router_w[l]);
+    a.router_b[l] = router_bias ? router_bias[l] : nullptr;
+  }
+  a.drafts = drafts;
+  a.argmax = argmax;
+  a.accepted = accepted;
+  a.out_tokens = out_tokens;
+  a.states = static_cast<__nv_bfloat16*>(states_out);
+  a.topk_idx = topk_idx_out;
+  a.part_gu = reinterpret_cast<float*>(ws + W.part_gu);
+  a.part_dn = reinterpret_cast<float*>(ws + W.part_dn);
+  a.act = reinterpret_cast<__nv_bfloat16*>(ws + W.act);
+  a.o = reinterpret_cast<__nv_bfloat16*>(ws + W.o);
+  a.ctrl = reinterpret_cast<SsCtrl*>(ws + W.ctrl);
+  if (cudaMemsetAsync(ws + W.ctrl, 0, sizeof(SsCtrl), s) != cudaSuccess) return cuda_fail();
+  ProfScope ps(VG_KERNEL_EXPERTS, s);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(dev->sms);
+  cfg.blockDim = dim3(kSsThreads);
+  cfg.dynamicSmemBytes = kSsSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, verify_step_small<kTopK>, maps, a) != cudaSuccess) return cuda_fail();
   return VG_OK;
 }

@@ -406,6 +406,39 @@ vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const void* x, con
                          void* kv_cache, const int32_t* lens, void* out, void* o_out, void* workspace,
                          size_t workspace_bytes, vg_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * The whole verify step for a handful of rows in ONE kernel launch: the
+ * n_layers MoE layers (x_{l+1} = bf16(x_l + MoE_l(x_l)), as vg_moe_ffn_stack),
+ * then the LM-head argmax and the prefix accept (as vg_verify_greedy). For
+ * T = B * (K+1) <= 16 rows (the batch-1 verify: K = 3 gives 4 rows, K = 1
+ * gives 2), where a step is a stream of weights and separate launches cost as
+ * much as the stream; the pages measure the speculative step at batch 1 and
+ * find launch overhead dominant there ("jina-ocr-v1: Schnellere
+ * Dokumentenanalyse auf kostengünstigen GPUs", "Spekulatives Decoding auf
+ * einer L4"). One CTA per SM (cooperative launch): every CTA computes the
+ * routing of all T rows itself (identical results, no barrier); the expert
+ * products are split along K over all SMs, and the pieces of a block are
+ * summed in k order by the last one to finish, so results do not depend on
+ * timing. The expert outputs differ from vg_moe_ffn_stack's only in the fp32
+ * summation order of the expert GEMMs.
+ * Arguments as vg_moe_ffn_stack (n_layers <= 12, bf16 pointers 16-byte
+ * aligned) and vg_verify_greedy (V >= 128); states_out, if not NULL, bf16
+ * [n_layers+1, T, H] receives each layer's input and then the final states;
+ * topk_idx_out, if not NULL, int32 [n_layers, T, 6] each layer's routed
+ * experts. workspace: vg_verify_step_small_workspace_bytes() bytes, 16-byte
+ * aligned, no initial contents (the call clears its control words first).
+ * B = 0 is a no-op. Errors: VG_ERR_INVALID_ARG, VG_ERR_UNSUPPORTED (T > 16,
+ * n_layers > 12, other dims, V < 128), VG_ERR_WORKSPACE, VG_ERR_CUDA; waits
+ * that run out record VG_ERR_TIMEOUT in the device status word.
+ * ------------------------------------------------------------------------- */
+size_t vg_verify_step_small_workspace_bytes(void);
+vg_status vg_verify_step_small(const vg_moe_dims* dims, int32_t n_layers, int32_t B, int32_t K, const void* x,
+                               const void* const* router_w, const float* const* router_bias,
+                               const void* const* expert_w, const void* const* shared_w, const void* lm_head,
+                               int32_t V, const int32_t* drafts, int32_t* argmax, int32_t* accepted,
+                               int32_t* out_tokens, void* states_out, int32_t* topk_idx_out, void* workspace,
+                               size_t workspace_bytes, vg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -206,3 +206,32 @@ def test_debug_wait_validation_before_launch(lib):
     assert f(vgv.VG_WAIT_MBARRIER, A, 61_000_000_000, None) == 1  # over a minute
     assert f(vgv.VG_WAIT_GRID_BARRIER, None, 1000, None) == 1     # the counter is needed
     assert f(vgv.VG_WAIT_GRID_BARRIER, A + 2, 1000, None) == 1    # misaligned counter
+
+
+def test_small_step_validation_before_launch(lib):
+    A = 1 << 40
+    need = lib.vg_verify_step_small_workspace_bytes()
+    assert need > 10 << 20
+    L = 12
+    arr = ctypes.c_void_p * L
+    w = arr(*[A + (i << 30) for i in range(L)])
+    d = ctypes.byref(vgv.MOE_DIMS)
+    f = lib.vg_verify_step_small
+
+    def call(n_layers=L, B=1, K=3, x=A, lm=A, V=129280, drafts=A, ws=A, n=need, rw=w, states=None, dims=d):
+        return f(dims, n_layers, B, K, x, rw, None, w, w, lm, V, drafts, A, A, A, states, None, ws, n, None)
+
+    assert call(B=0) == 0                       # no-op
+    assert call(B=-1) == 1
+    assert call(n_layers=0) == 1
+    assert call(n_layers=13) == 2               # at most 12 layers
+    assert call(B=5, K=3) == 2                  # 20 rows > 16
+    assert call(x=None) == 1
+    assert call(drafts=None) == 1               # drafts needed when K > 0
+    assert call(x=A + 8) == 1                   # misaligned
+    assert call(states=A + 8) == 1
+    assert call(rw=None) == 1
+    assert call(n=need - 1) == 3
+    assert call(ws=A + 8) == 3
+    assert call(dims=ctypes.byref(vgv.vg_moe_dims(1280, 896, 64, 2, 8))) == 2
+
