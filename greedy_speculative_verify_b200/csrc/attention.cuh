@@ -14,9 +14,9 @@
 //   exp-weighted value sum for each new row; every key and value of the chunk
 //   is read once for all K+1 rows, both products on the tensor cores.
 // attn_merge: merges a (sequence, head, row)'s chunk partials into o.
-// attn_proj_splitk: the q/k/v and output projections as fp32 partial sums over
-//   256-wide slices of the reduction, summed in a fixed order by their readers
-//   (attn_rope_append, attn_residual), which round the sum to bf16.
+// The q/k/v and output projections are fp32 partial sums over 256-wide slices
+// of the reduction (attn_proj_tc, proj_tc.cuh), summed in a fixed order by
+// their readers (attn_rope_append, attn_residual), which round the sum to bf16.
 #pragma once
 #include "common.cuh"
 
@@ -25,8 +25,8 @@ namespace vg {
 constexpr int kAttnHeads = 10, kAttnDim = 128;
 constexpr int kAttnChunk = 256;   // cache positions per CTA
 constexpr int kAttnMaxRows = 8;   // K + 1 <= 8 new rows per sequence
-constexpr int kAttnThreads = 256;
-constexpr int kProjN = 64, kProjK = 256, kProjM = 128;  // projection block: outputs, reduction slice, rows
+constexpr int kAttnThreads = 256; // 8 warps of 32 positions
+
 
 struct AttnArgs {
   int32_t B, K1, L_max;          // K1 = K + 1 rows per sequence
@@ -54,52 +54,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// part[s][r][n] = sum over k in [256 s, 256 s + 256) of x[r][k] W[n][k] (fp32),
-// for x bf16 [R, K] and W bf16 [N, K] (N a multiple of 64, K of 256).
-// grid (N / 64, K / 256, cdiv(R, 128)), 256 threads: warp w takes rows
-// 128 z + 16 w .. +15 against the block's 64 outputs (8 tensor-core n-tiles).
-// A lane loads 16 contiguous bytes of a row of x and of W per 32-wide step of
-// the reduction; both operands take the same order of k inside the step, so
-// the sum is unchanged. The reduction is split so that a launch has
-// N / 64 x K / 256 blocks streaming the weights (60 x 5 for q/k/v).
-__global__ void __launch_bounds__(256) attn_proj_splitk(const __nv_bfloat16* __restrict__ x,
-                                                        const __nv_bfloat16* __restrict__ w, int R, int N, int K,
-                                                        float* __restrict__ part) {
-  griddep_launch_dependents();
-  griddep_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int n0 = blockIdx.x * kProjN, sl = blockIdx.y, k0 = sl * kProjK;
-  const int r0 = blockIdx.z * kProjM + 16 * warp;
-  if (r0 >= R) return;  // the whole warp: rows past the end
-  const int ra = r0 + g, rb = r0 + g + 8;
-  const uint4 zero4 = make_uint4(0, 0, 0, 0);
-  const __nv_bfloat16* xa = x + (size_t)ra * K + k0 + 8 * t;
-  const __nv_bfloat16* xb = x + (size_t)rb * K + k0 + 8 * t;
-  const __nv_bfloat16* wr = w + (size_t)(n0 + g) * K + k0 + 8 * t;
-  float acc[kProjN / 8][4];
-#pragma unroll
-  for (int j = 0; j < kProjN / 8; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
-#pragma unroll 2
-  for (int q = 0; q < kProjK / 32; ++q) {
-    const uint4 av = ra < R ? __ldg(reinterpret_cast<const uint4*>(xa + 32 * q)) : zero4;
-    const uint4 bv = rb < R ? __ldg(reinterpret_cast<const uint4*>(xb + 32 * q)) : zero4;
-#pragma unroll
-    for (int j = 0; j < kProjN / 8; ++j) {
-      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + (size_t)8 * j * K + 32 * q));
-      mma_16816(acc[j], av.x, bv.x, av.y, bv.y, wv.x, wv.y);
-      mma_16816(acc[j], av.z, bv.z, av.w, bv.w, wv.z, wv.w);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kProjN / 8; ++j) {
-    const int n = n0 + 8 * j + 2 * t;
-    if (ra < R) *reinterpret_cast<float2*>(part + ((size_t)sl * R + ra) * N + n) = make_float2(acc[j][0], acc[j][1]);
-    if (rb < R) *reinterpret_cast<float2*>(part + ((size_t)sl * R + rb) * N + n) = make_float2(acc[j][2], acc[j][3]);
-  }
 }
 
 // bf16 of the fixed-order sum of `splits` partials p[0], p[stride], ...
@@ -180,13 +134,14 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
   return d;
 }
 
-// grid (B * heads, n_chunks), 256 threads; warp w takes positions 32w .. 32w+31
-// of the chunk, lane = (g, t) = (lane / 4, lane % 4), the K+1 <= 8 new rows as
-// rows 0..7 of 16-row tensor-core tiles (rows 8..15 zero).
+// grid (B * heads, n_chunks), 256 threads, two CTAs per SM; warp w takes
+// positions 32w .. 32w+31 of the chunk, lane = (g, t) = (lane / 4, lane % 4),
+// the K+1 <= 8 new rows as rows 0..7 of 16-row tensor-core tiles (rows 8..15
+// zero).
 //   scores: S = Q K^T over 8 positions per tile; a lane loads 16 contiguous
-//     bytes (dimensions 32s + 8t .. +7 of one key, s = 0..3), giving the B
-//     operands of two k-steps; the queries are loaded with the same dimension
-//     order, so the contraction is unchanged;
+//     bytes of one key from global memory (dimensions 32s + 8t .. +7, s =
+//     0..3), giving the B operands of two k-steps; the queries are loaded with
+//     the same dimension order, so the contraction is unchanged;
 //   softmax over the warp's 32 positions, per row: max and the exp-weights,
 //     rounded to bf16 pairs that are already the A operand of the next product
 //     (the exp-sum is taken over the rounded weights);
@@ -195,145 +150,152 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
 //     ends with dimensions 32s + 8t .. +7 of row g;
 //   the 8 warps' (max, exp-sum, values) are merged in shared memory into the
 //     chunk's partial.
+// Positions past the visible ones read as zero keys and values. (Staging the
+// keys and values through shared memory with TMA measured slower for this
+// access pattern, a 256-byte piece of every 2,560-byte cache row, than these
+// 16-byte loads from all 256 threads; so did merging the partials in the last
+// CTA of each (sequence, head), whose fence and counter lengthen every CTA.)
 __global__ void __launch_bounds__(kAttnThreads, 2) attn_chunk(const AttnArgs a) {
-  griddep_launch_dependents();
-  griddep_wait();
   constexpr int H = kAttnHeads * kAttnDim;
   constexpr int PW = 2 + kAttnDim;  // floats per row of a partial
   constexpr int OW = kAttnDim + 4;  // padded row of the per-warp values
-  static_assert(kAttnMaxRows <= 8 && kAttnThreads == 256 && kAttnDim == 128 && kAttnChunk == 256,
-                "the lane maps below assume 8 warps of 32 positions, 128 dimensions, at most 8 rows");
-  __shared__ float wm[8][8], wl[8][8];              // per warp and row: max, exp-sum
-  __shared__ __align__(16) float wo[8][8][OW];      // per warp and row: exp-weighted values
+  constexpr int NW = kAttnThreads / 32;
+  static_assert(kAttnMaxRows <= 8 && NW * 32 == kAttnChunk && kAttnDim == 128,
+                "the lane maps below assume warps of 32 positions, 128 dimensions, at most 8 rows");
+  __shared__ float wm[NW][8], wl[NW][8];            // per warp and row: max, exp-sum
+  __shared__ __align__(16) float wo[NW][8][OW];     // per warp and row: exp-weighted values
   const int b = blockIdx.x / kAttnHeads, h = blockIdx.x - b * kAttnHeads, c = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int K1 = a.K1;
+  griddep_launch_dependents();
+  griddep_wait();  // the rotated queries and the new keys and values come from the previous kernel
   int L;
   const bool ok = attn_len_ok(a, b, &L);
   const int visible = ok ? L + K1 : 0;  // positions any row of this step may see
   const int p0 = c * kAttnChunk, n = max(0, min(kAttnChunk, visible - p0));
   float* part = a.part + (((size_t)b * kAttnHeads + h) * a.n_chunks + c) * K1 * PW;
-  if (n == 0) {  // nothing here: an empty partial
+  if (n > 0) {
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+    const int wp = 32 * warp;  // the warp's first position in the chunk
+    // ---- scores
+    uint4 qf[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      qf[s] = g < K1 ? *reinterpret_cast<const uint4*>(a.q + ((size_t)b * K1 + g) * H + h * kAttnDim + 32 * s + 8 * t)
+                     : zero4;
+    const __nv_bfloat16* kb = a.cache + ((size_t)b * 2 * a.L_max + p0 + wp) * H + h * kAttnDim + 8 * t;
+    float sc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int pos = 8 * j + g;  // the key this lane loads
+      uint4 kf[4];
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        kf[s] = wp + pos < n ? __ldg(reinterpret_cast<const uint4*>(kb + (size_t)pos * H + 32 * s)) : zero4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[j][e] = 0.0f;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        mma_16816_top(sc[j], qf[s].x, qf[s].y, kf[s].x, kf[s].y);
+        mma_16816_top(sc[j], qf[s].z, qf[s].w, kf[s].z, kf[s].w);
+      }
+    }
+    // ---- softmax of row g over the warp's positions (lanes 4g .. 4g+3 share the row)
+    const float scale = 1.0f / sqrtf((float)kAttnDim);
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int pos = wp + 8 * j + 2 * t + e;
+        const bool seen = g < K1 && pos < n && p0 + pos <= L + g;  // causal
+        sc[j][e] = seen ? sc[j][e] * scale : -INFINITY;
+        m = fmaxf(m, sc[j][e]);
+      }
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    uint32_t pf[4];  // exp-weights of positions 8j + 2t, 8j + 2t + 1 as bf16 pairs
+    float l = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float e0 = sc[j][0] == -INFINITY ? 0.0f : expf(sc[j][0] - m);
+      const float e1 = sc[j][1] == -INFINITY ? 0.0f : expf(sc[j][1] - m);
+      const __nv_bfloat162 pp = __floats2bfloat162_rn(e0, e1);
+      pf[j] = *reinterpret_cast<const uint32_t*>(&pp);
+      l += __low2float(pp) + __high2float(pp);
+    }
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    // ---- values: O = P V over the warp's positions, two k-steps of 16
+    float o[4][4][4];  // [dimension block s][tile j][accumulator]: row g, dimensions 32s + 8t + 2j + {0, 1}
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[s][j][e] = 0.0f;
+    const __nv_bfloat16* vb = a.cache + ((size_t)(b * 2 + 1) * a.L_max + p0 + wp) * H + h * kAttnDim + 8 * t;
+#pragma unroll
+    for (int kp = 0; kp < 2; ++kp) {
+      const int lo = 16 * kp + g, hi = lo + 8;  // the value rows this lane reads
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint4 vl = wp + lo < n ? __ldg(reinterpret_cast<const uint4*>(vb + (size_t)lo * H + 32 * s)) : zero4;
+        const uint4 vh = wp + hi < n ? __ldg(reinterpret_cast<const uint4*>(vb + (size_t)hi * H + 32 * s)) : zero4;
+        const uint32_t rl[4] = {vl.x, vl.y, vl.z, vl.w}, rh[4] = {vh.x, vh.y, vh.z, vh.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_16816_top(o[s][j], pf[2 * kp], pf[2 * kp + 1], movmatrix_trans(rl[j]), movmatrix_trans(rh[j]));
+      }
+    }
+    // ---- merge the warps into the chunk's partial
+    if (t == 0) {
+      wm[warp][g] = m;
+      wl[warp][g] = l;
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      float* dst = &wo[warp][g][32 * s + 8 * t];
+      *reinterpret_cast<float4*>(dst) = make_float4(o[s][0][0], o[s][0][1], o[s][1][0], o[s][1][1]);
+      *reinterpret_cast<float4*>(dst + 4) = make_float4(o[s][2][0], o[s][2][1], o[s][3][0], o[s][3][1]);
+    }
+    __syncthreads();
+    for (int i = tid; i < K1 * (kAttnDim / 4); i += kAttnThreads) {
+      const int r = i / (kAttnDim / 4), d4 = 4 * (i % (kAttnDim / 4));
+      float mm = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) mm = fmaxf(mm, wm[w][r]);
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      float ls = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        if (wm[w][r] == -INFINITY) continue;  // no visible position in that warp's share
+        const float f = expf(wm[w][r] - mm);
+        ls = __fmaf_rn(wl[w][r], f, ls);
+        const float4 v = *reinterpret_cast<const float4*>(&wo[w][r][d4]);
+        acc.x = __fmaf_rn(v.x, f, acc.x);
+        acc.y = __fmaf_rn(v.y, f, acc.y);
+        acc.z = __fmaf_rn(v.z, f, acc.z);
+        acc.w = __fmaf_rn(v.w, f, acc.w);
+      }
+      float* pr = part + (size_t)r * PW;
+      pr[2 + d4] = acc.x;
+      pr[3 + d4] = acc.y;
+      pr[4 + d4] = acc.z;
+      pr[5 + d4] = acc.w;
+      if (d4 == 0) {
+        pr[0] = mm;
+        pr[1] = ls;
+      }
+    }
+  } else {  // nothing visible here: an empty partial
     for (int i = tid; i < K1; i += blockDim.x) {
       part[(size_t)i * PW] = -INFINITY;
       part[(size_t)i * PW + 1] = 0.0f;
     }
     for (int i = tid; i < K1 * kAttnDim; i += blockDim.x) part[(size_t)(i / kAttnDim) * PW + 2 + i % kAttnDim] = 0.0f;
-    return;
   }
-  const uint4 zero4 = make_uint4(0, 0, 0, 0);
-  const int wp = 32 * warp;  // the warp's first position in the chunk
-  // ---- scores
-  uint4 qf[4];
-#pragma unroll
-  for (int s = 0; s < 4; ++s)
-    qf[s] = g < K1 ? *reinterpret_cast<const uint4*>(a.q + ((size_t)b * K1 + g) * H + h * kAttnDim + 32 * s + 8 * t)
-                   : zero4;
-  const __nv_bfloat16* kb = a.cache + ((size_t)b * 2 * a.L_max + p0 + wp) * H + h * kAttnDim + 8 * t;
-  float sc[4][4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int pos = 8 * j + g;  // the key this lane loads
-    uint4 kf[4];
-#pragma unroll
-    for (int s = 0; s < 4; ++s)
-      kf[s] = wp + pos < n ? __ldg(reinterpret_cast<const uint4*>(kb + (size_t)pos * H + 32 * s)) : zero4;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sc[j][e] = 0.0f;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      mma_16816_top(sc[j], qf[s].x, qf[s].y, kf[s].x, kf[s].y);
-      mma_16816_top(sc[j], qf[s].z, qf[s].w, kf[s].z, kf[s].w);
-    }
-  }
-  // ---- softmax of row g over the warp's positions (lanes 4g .. 4g+3 share the row)
-  const float scale = 1.0f / sqrtf((float)kAttnDim);
-  float m = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int pos = wp + 8 * j + 2 * t + e;
-      const bool seen = g < K1 && pos < n && p0 + pos <= L + g;  // causal
-      sc[j][e] = seen ? sc[j][e] * scale : -INFINITY;
-      m = fmaxf(m, sc[j][e]);
-    }
-  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-  uint32_t pf[4];  // exp-weights of positions 8j + 2t, 8j + 2t + 1 as bf16 pairs
-  float l = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float e0 = sc[j][0] == -INFINITY ? 0.0f : expf(sc[j][0] - m);
-    const float e1 = sc[j][1] == -INFINITY ? 0.0f : expf(sc[j][1] - m);
-    const __nv_bfloat162 pp = __floats2bfloat162_rn(e0, e1);
-    pf[j] = *reinterpret_cast<const uint32_t*>(&pp);
-    l += __low2float(pp) + __high2float(pp);
-  }
-  l += __shfl_xor_sync(0xffffffffu, l, 1);
-  l += __shfl_xor_sync(0xffffffffu, l, 2);
-  // ---- values: O = P V over the warp's positions, two k-steps of 16
-  float o[4][4][4];  // [dimension block s][tile j][accumulator]: row g, dimensions 32s + 8t + 2j + {0, 1}
-#pragma unroll
-  for (int s = 0; s < 4; ++s)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[s][j][e] = 0.0f;
-  const __nv_bfloat16* vb = a.cache + ((size_t)(b * 2 + 1) * a.L_max + p0 + wp) * H + h * kAttnDim + 8 * t;
-#pragma unroll
-  for (int kp = 0; kp < 2; ++kp) {
-    const int lo = 16 * kp + g, hi = lo + 8;  // the value rows this lane loads
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const uint4 vl = wp + lo < n ? __ldg(reinterpret_cast<const uint4*>(vb + (size_t)lo * H + 32 * s)) : zero4;
-      const uint4 vh = wp + hi < n ? __ldg(reinterpret_cast<const uint4*>(vb + (size_t)hi * H + 32 * s)) : zero4;
-      const uint32_t rl[4] = {vl.x, vl.y, vl.z, vl.w}, rh[4] = {vh.x, vh.y, vh.z, vh.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        mma_16816_top(o[s][j], pf[2 * kp], pf[2 * kp + 1], movmatrix_trans(rl[j]), movmatrix_trans(rh[j]));
-    }
-  }
-  // ---- merge the 8 warps into the chunk's partial
-  if (t == 0) {
-    wm[warp][g] = m;
-    wl[warp][g] = l;
-  }
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    float* dst = &wo[warp][g][32 * s + 8 * t];
-    *reinterpret_cast<float4*>(dst) = make_float4(o[s][0][0], o[s][0][1], o[s][1][0], o[s][1][1]);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(o[s][2][0], o[s][2][1], o[s][3][0], o[s][3][1]);
-  }
-  __syncthreads();
-  for (int i = tid; i < K1 * (kAttnDim / 4); i += kAttnThreads) {
-    const int r = i / (kAttnDim / 4), d4 = 4 * (i % (kAttnDim / 4));
-    float mm = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, wm[w][r]);
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    float ls = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      if (wm[w][r] == -INFINITY) continue;  // no visible position in that warp's share
-      const float f = expf(wm[w][r] - mm);
-      ls = __fmaf_rn(wl[w][r], f, ls);
-      const float4 v = *reinterpret_cast<const float4*>(&wo[w][r][d4]);
-      acc.x = __fmaf_rn(v.x, f, acc.x);
-      acc.y = __fmaf_rn(v.y, f, acc.y);
-      acc.z = __fmaf_rn(v.z, f, acc.z);
-      acc.w = __fmaf_rn(v.w, f, acc.w);
-    }
-    float* pr = part + (size_t)r * PW;
-    pr[2 + d4] = acc.x;
-    pr[3 + d4] = acc.y;
-    pr[4 + d4] = acc.z;
-    pr[5 + d4] = acc.w;
-    if (d4 == 0) {
-      pr[0] = mm;
-      pr[1] = ls;
-    }
-  }
+
 }
 
 // grid B * heads * K1, kAttnDim threads: o = sum_c acc_c e^(m_c - m) / sum_c l_c e^(m_c - m).
@@ -358,5 +320,6 @@ __global__ void __launch_bounds__(kAttnDim) attn_merge(const AttnArgs a) {
   }
   a.o[((size_t)b * a.K1 + r) * H + h * kAttnDim + d] = __float2bfloat16_rn(l > 0.0f ? acc / l : 0.0f);
 }
+
 
 }  // namespace vg

@@ -14,6 +14,7 @@
 #include "decode_loop.cuh"
 #include "mtp.cuh"
 #include "attention.cuh"
+#include "proj_tc.cuh"
 #include "gemm_moe.cuh"
 #include "gemm_tm.cuh"
 #include "layer_entry.cuh"
@@ -137,6 +138,9 @@ vg_status device_state(DevState** out) {
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::verify_step_small<kTopK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vg::kSsSmemBytes) != cudaSuccess)
+      return cuda_fail();
+    if (cudaFuncSetAttribute(vg::attn_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kPtSmemBytes) !=
+            cudaSuccess)
       return cuda_fail();
     if (cudaFuncSetAttribute(vg::lmhead_argmax_accept, cudaFuncAttributeMaxDynamicSharedMemorySize, vg::kLmSmemBytes) !=
         cudaSuccess)
@@ -1091,7 +1095,7 @@ namespace {
 struct AttnWs {
   size_t pk, q, o, part, total;
 };
-constexpr int kProjSplits = kH / vg::kProjK;  // partial sums of a projection (5)
+constexpr int kProjSplits = kH / vg::kPtK;  // partial sums of a projection (5)
 AttnWs attn_layout(int B, int K, int L_max) {
   const size_t R = (size_t)B * (K + 1);
   AttnWs L{};
@@ -1121,8 +1125,9 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   using namespace vg;
   if (B < 0 || K < 0 || K + 1 > kAttnMaxRows || L_max < 1 || L_max > 32768) return VG_ERR_INVALID_ARG;
   if (B == 0) return VG_OK;
-  // launch sizes count (row, head-pair) items in int
-  if ((int64_t)B * (K + 1) * kH >= ((int64_t)1 << 31)) return VG_ERR_UNSUPPORTED;
+  // launch sizes count (row, head-pair) items and the cache's rows in int
+  if ((int64_t)B * (K + 1) * kH >= ((int64_t)1 << 31) || (int64_t)B * 2 * L_max >= ((int64_t)1 << 31))
+    return VG_ERR_UNSUPPORTED;
   if (!x || !w_qkv || !w_o || !kv_cache || !lens || !out) return VG_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(w_o) || !aligned16(kv_cache) || !aligned16(out) ||
       !aligned16(o_out))
@@ -1142,19 +1147,23 @@ extern "C" vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const v
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(ws + o); };
   float* pk = reinterpret_cast<float*>(ws + L.pk);
-  const int mblocks = cdiv(R, kProjM);
+  // x W^T as fp32 partial sums over the 5 slices of the reduction, on the tensor cores
   auto launch_proj = [&](const void* act, const void* wgt, int n_out) {
-    cudaLaunchConfig_t pc = {};  // 3-d grid: (64 outputs, 256-wide reduction slice, 128 rows)
-    pc.gridDim = dim3(n_out / kProjN, kProjSplits, mblocks);
-    pc.blockDim = dim3(256);
+    CUtensorMap mW, mX;
+    const uint64_t dW[2] = {kH, (uint64_t)n_out}, dX[2] = {kH, (uint64_t)R}, sK[1] = {kH * 2};
+    const uint32_t bW[2] = {kBK, kBM}, bX[2] = {kBK, (uint32_t)box_rows(R, kPtRows)};
+    if (make_map(&mW, wgt, 2, dW, sK, bW) || make_map(&mX, act, 2, dX, sK, bX)) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t pc = {};  // 3-d grid: (128 outputs, 256-wide reduction slice, 128 rows)
+    pc.gridDim = dim3(n_out / kBM, kProjSplits, cdiv(R, kPtRows));
+    pc.blockDim = dim3(192);
+    pc.dynamicSmemBytes = kPtSmemBytes;
     pc.stream = s;
     cudaLaunchAttribute pa[1];
     pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pa[0].val.programmaticStreamSerializationAllowed = 1;
     pc.attrs = pa;
     pc.numAttrs = 1;
-    return cudaLaunchKernelEx(&pc, attn_proj_splitk, static_cast<const __nv_bfloat16*>(act),
-                              static_cast<const __nv_bfloat16*>(wgt), R, n_out, (int)kH, pk);
+    return cudaLaunchKernelEx(&pc, attn_proj_tc, mW, mX, R, n_out, (int)bX[1], pk);
   };
   // q/k/v = x W_qkv^T as split partial sums
   if (launch_proj(x, w_qkv, 3 * kH) != cudaSuccess) return cuda_fail();

@@ -397,9 +397,13 @@ vg_status vg_mtp_draft(int32_t B, int32_t K, const vg_mtp_weights* w, const void
  * them kv_cache. Precision: both products of a head (q.k and the
  * probability-weighted sum of v) run on the tensor cores with bf16 operands and
  * fp32 accumulation, so the softmax weights enter the second product rounded to
- * bf16 (their sum is taken over the rounded weights). Errors: VG_ERR_INVALID_ARG,
- * VG_ERR_UNSUPPORTED (B*(K+1)*H >= 2^31), VG_ERR_WORKSPACE (null, short or not
- * 16-byte aligned), VG_ERR_CUDA.
+ * bf16 (their sum is taken over the rounded weights); the projections run on
+ * the tcgen05 tensor cores as fp32 sums over five 256-wide slices of the
+ * reduction, added in slice order. Six launches: q/k/v projection, rotary
+ * append, attention over 256-position chunks, the merge of the chunks, output
+ * projection, residual. Errors: VG_ERR_INVALID_ARG, VG_ERR_UNSUPPORTED
+ * (B*(K+1)*H >= 2^31 or B*2*L_max >= 2^31), VG_ERR_WORKSPACE (null, short or
+ * not 16-byte aligned), VG_ERR_CUDA.
  * ------------------------------------------------------------------------- */
 size_t vg_attn_workspace_bytes(int32_t B, int32_t K, int32_t L_max);
 vg_status vg_attn_verify(int32_t B, int32_t K, int32_t L_max, const void* x, const void* w_qkv, const void* w_o,
