@@ -48,10 +48,17 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
+DEBUG_LIB = os.path.join(PKG, "libvgv_debug.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None, out: str | None = None) -> str:
+    """Builds the library (out=None: LIB, skipped when up to date). out names
+    another file, e.g. DEBUG_LIB with extra_flags=["-DVG_DEBUG_BOUNDS"]."""
+    target = out or LIB
+    if not force and (up_to_date() if out is None else
+                      os.path.exists(target) and all(os.path.getmtime(s) <= os.path.getmtime(target) for s in sources())):
+        return target
+    tmp = target + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
            "-o", tmp, os.path.join(CSRC, "vgv_api.cu")]
     if verbose:
@@ -61,8 +68,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if verbose and (r.stdout or r.stderr):
         print(r.stdout, r.stderr, sep="\n")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

@@ -22,6 +22,7 @@ __device__ __forceinline__ uint4 combine8(const __nv_bfloat16* __restrict__ x, c
   }
   for (int j = 0; j < k; ++j) {
     const int p = inv[t * k + j];
+    if (!VG_IN_BOUNDS((unsigned)p < (unsigned)(k * T), 401)) continue;
     const float gj = g[t * k + j];
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(o + (size_t)p * H) + c);
     y[0] = __fmaf_rn(gj, bf16_lo(v.x), y[0]); y[1] = __fmaf_rn(gj, bf16_hi(v.x), y[1]);

@@ -23,6 +23,16 @@ __device__ __forceinline__ void record_error(int32_t code, int32_t site) {
   if (atomicCAS(&g_status, 0, code) == 0) atomicExch(&g_status_info, site);
 }
 
+// Checks of computed indices, compiled in with -DVG_DEBUG_BOUNDS (the debug
+// build, a stand-in for a memory checker): a failed check records
+// VG_ERR_DEVICE_BOUNDS with its site and the guarded access is skipped. In the
+// normal build the macro is the constant true and the checks vanish.
+#ifdef VG_DEBUG_BOUNDS
+#define VG_IN_BOUNDS(cond, site) ((cond) ? true : (::vg::record_error(::vg::kErrBounds, (site)), false))
+#else
+#define VG_IN_BOUNDS(cond, site) true
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

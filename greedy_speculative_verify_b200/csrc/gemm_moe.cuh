@@ -487,6 +487,9 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
+      // the unit's rows lie inside the activation / output buffers: routed rows, then S x T shared rows
+      const bool rows_ok = VG_IN_BOUNDS(un.arow >= 0 && un.arow + un.nrows <= sch->arow[args.E] + args.S * args.T,
+                                        404);
       const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + ab * C::kAccCols;
       if (un.down) {
         const int ld = args.mblk_dn * 2 * kBM;
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (c0 + j < un.nrows) {
+            if (rows_ok && c0 + j < un.nrows) {
               dst[(size_t)(c0 + j) * ld] = __float2bfloat16_rn(__uint_as_float(g[j]));
               dst[(size_t)(c0 + j) * ld + kBM] = __float2bfloat16_rn(__uint_as_float(v[j]));
             }
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (c0 + j < un.nrows)
+            if (rows_ok && c0 + j < un.nrows)
               dst[(size_t)(c0 + j) * ld] = __float2bfloat16_rn(silu(__uint_as_float(g[j])) * __uint_as_float(v[j]));
         }
       }

@@ -311,8 +311,11 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
+      // the unit's rows lie inside the activation / output buffers: routed rows, then S x T shared rows
+      const bool rows_ok = VG_IN_BOUNDS(un.arow >= 0 && un.arow + un.nrows <= sch->arow[args.E] + args.S * args.T,
+                                        406);
       const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + ab * kTmAccCols;
-      const bool mine = row < un.nrows;
+      const bool mine = rows_ok && row < un.nrows;
       if (un.down) {
         const int ld = args.mblk_dn * kTmN;
         uint4* dst = reinterpret_cast<uint4*>(args.out + (size_t)(un.arow + row) * ld + un.mb * kTmN);

@@ -314,13 +314,18 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
     int rank = 0;
     for (int j2 = 0; j2 < tid; ++j2) rank += idx_s[j2] == key;
     my_pos = off_s[key] + pre_s[key] + rank;
-    a.perm[my_pos] = a_begin + tid;
-    a.inv[a_begin + tid] = my_pos;
+    if (VG_IN_BOUNDS((unsigned)my_pos < (unsigned)N && a_begin + tid < N, 402)) {
+      a.perm[my_pos] = a_begin + tid;
+      a.inv[a_begin + tid] = my_pos;
+    } else {
+      my_pos = -1;
+    }
   }
   __syncthreads();  // every rank was taken from idx_s before it is overwritten
   if (tid < n_own * K) idx_s[tid] = my_pos;
   __syncthreads();
   for (int i = warp; i < n_own * K; i += blockDim.x / 32) {
+    if (!VG_IN_BOUNDS((unsigned)idx_s[i] < (unsigned)N, 403)) continue;
     const uint4* src = reinterpret_cast<const uint4*>(xo + (size_t)(i / K) * H);
     uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (size_t)idx_s[i] * H);
     for (int cc = lane; cc < H / 8; cc += 32) dst[cc] = src[cc];

@@ -279,7 +279,8 @@ __global__ void __launch_bounds__(192, 1)
   __threadfence();
   for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
     const unsigned long long k = atomicExch(a.best + r, 0ull);
-    a.argmax[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    const int32_t v = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    a.argmax[r] = VG_IN_BOUNDS(v >= 0 && v < a.V, 409) ? v : 0;
   }
   __syncthreads();  // every argmax of this CTA is visible to all its threads
   for (int b = threadIdx.x; b < a.B; b += blockDim.x) {

@@ -134,8 +134,9 @@ __global__ void __launch_bounds__(1024) expert_scatter_chunks(const int32_t* __r
   if (tid < kSortE) run[tid] = chunk_base[blockIdx.x * kSortE + tid];
   __syncthreads();
   const int base = blockIdx.x * kSortChunk;
-  const int pos = chunk_positions(keys, base, N, run, wcnt);
+  int pos = chunk_positions(keys, base, N, run, wcnt);
   const int a = base + tid;
+  if (pos >= 0 && !VG_IN_BOUNDS(pos < N, 408)) pos = -1;
   pos_s[tid] = pos;
   if (pos >= 0) {
     perm[pos] = a;

@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(kSsThreads, 1)
         }
         for (int j = 0; j < K6; ++j) {
           const float gj = g_s[t][j];
+          if (!VG_IN_BOUNDS((unsigned)sl_s[t][j] < (unsigned)kSsSlots, 411)) continue;
           const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.o + ((size_t)sl_s[t][j] * kSsN + t) * H) + c8);
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -682,7 +683,8 @@ __global__ void __launch_bounds__(kSsThreads, 1)
   __threadfence();
   for (int t = tid; t < T; t += kSsThreads) {
     const unsigned long long k = atomicExch(&a.ctrl->best[t], 0ull);
-    a.argmax[t] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    const int32_t v = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    a.argmax[t] = VG_IN_BOUNDS(v >= 0 && v < a.V, 410) ? v : 0;
   }
   __syncthreads();
   for (int b = tid; b < a.B; b += kSsThreads) {

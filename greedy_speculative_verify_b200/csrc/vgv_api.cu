@@ -302,8 +302,15 @@ bool static_first_units(const DevState* dev, int T) {
 
 // The layer-entry kernel takes decode sizes: at most kEntryMaxOwn tokens per CTA
 // of its cooperative grid.
+#ifndef VG_ENTRY_TOK_PER_CTA
+#define VG_ENTRY_TOK_PER_CTA 1
+#endif
 int entry_grid(const DevState* dev, int T) {
-  return std::min(std::min(std::min(dev->sms, kEntryMaxGrid), vg::kEntryMaxGridDev), T);
+  const int g = std::min(std::min(std::min(dev->sms, kEntryMaxGrid), vg::kEntryMaxGridDev), T);
+  // with fixed first units the expert kernel's CTAs stream weights on every SM
+  // the entry leaves free, so the entry may take several tokens per CTA
+  const int per = T >= kStaticFirstMinT ? VG_ENTRY_TOK_PER_CTA : 1;
+  return std::max(1, std::min(g, vg::cdiv(T, per)));
 }
 bool small_path(const DevState* dev, int T) {
   return (int64_t)T * kTopK <= vg::kSortSmallMax && vg::cdiv(T, entry_grid(dev, T)) <= vg::kEntryMaxOwn;

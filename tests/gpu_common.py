@@ -11,6 +11,8 @@ Comparison rules (the tolerances of the parity bar):
   z64 the fp64 logit and A = sum_h |hid_h * LM_vh|, a bound on the error of any
   fp32 summation order over 1280 terms.
 """
+import os
+
 import numpy as np
 import torch
 
@@ -25,7 +27,12 @@ TIE_EPS = 2.0 ** -14
 
 
 def ensure_lib():
+    """Builds and loads the library; VG_TEST_LIB names another build of it to
+    test instead (the bounds-checking debug build, tests/test_gpu_zy_debug_bounds.py)."""
     vbuild.build()
+    other = os.environ.get("VG_TEST_LIB")
+    if other:
+        vgv.LIB_PATH = other
     vgv.load()
 
 
