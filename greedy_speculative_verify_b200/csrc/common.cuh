@@ -285,7 +285,11 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* ctr, uint32_t target, uin
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    __threadfence();  // this CTA's writes (ordered before by __syncthreads) precede the arrival
+    // release: this CTA's writes, ordered before it by the __syncthreads above,
+    // are visible to every CTA whose acquire below reads the final count
+#ifdef VG_GRID_BARRIER_FENCES
+    __threadfence();
+#endif
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
     const uint64_t t0 = globaltimer();
     while (true) {
@@ -298,8 +302,10 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* ctr, uint32_t target, uin
         break;
       }
     }
+#ifdef VG_GRID_BARRIER_FENCES
     __threadfence();
-    ok_s = ok;
+#endif
+    ok_s = ok;  // the __syncthreads below passes the acquire on to the whole CTA
   }
   __syncthreads();
   return ok_s != 0;

@@ -52,9 +52,13 @@ constexpr int kMaxExperts = 72;
 //    small and the freed shared memory buys a fifth stage of weights in flight;
 //  * NMAX = 16, 6 stages: a handful of tokens (batch-1 verify), where every
 //    expert's tokens fit one 16-row tile and a sixth stage fits.
+#ifndef VG_FG_STAGES_64
+#define VG_FG_STAGES_64 5
+#endif
+
 template <int NMAX>
 struct FgCfg {
-  static constexpr int kStages = NMAX == 128 ? 4 : NMAX == 64 ? 5 : 6;
+  static constexpr int kStages = NMAX == 128 ? 4 : NMAX == 64 ? VG_FG_STAGES_64 : 6;
   static constexpr int kABytes = 2 * kBM * kBK * 2;      // two 16 KB weight tiles
   static constexpr int kBBytes = NMAX * kBK * 2;         // token slot
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -81,7 +85,11 @@ struct FusedArgs {
   // 1: every expert has a primary tile (its first NMAX tokens, possibly none),
   // tiles 0 .. E+S-1 in expert order, then the further tiles; CTA b's first unit
   // is unit b (a gate/up unit of a primary tile, known before the routing), and
-  // its weights are requested before the kernel waits for the previous one
+  // its weights are requested before the kernel waits for the previous one.
+  // The gate/up token rows of routed expert e's primary tile are rows
+  // e NMAX .. e NMAX + NMAX - 1 of the B map, its further tiles' rows follow
+  // E NMAX + (segment offset), so the first unit's token rows are requested
+  // right after the wait, before the offsets are read
   int32_t static_first;
   int32_t pre_l2_chunks;   // static_first: k-chunks of the first unit past the stages, prefetched to L2
 };
@@ -131,7 +139,7 @@ __device__ __forceinline__ FgUnit fg_decode(int u, const FgSched& s, int n_exp, 
   }
   un.e = e;
   un.nrows = max(0, min(nmax, s.n[e] - nb * nmax));  // 0 only for the primary tile of an expert without tokens
-  un.xrow = s.xrow[e] + nb * nmax;
+  un.xrow = a.static_first && nb == 0 && e < a.E ? e * nmax : s.xrow[e] + nb * nmax;
   un.arow = s.arow[e] + nb * nmax;
   return un;
 }
@@ -166,6 +174,7 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);  // kFgRing tickets
+  uint64_t* sched_ready = reinterpret_cast<uint64_t*>(aux + 256);        // the schedule below is built
   FgSched* sch = reinterpret_cast<FgSched*>(aux + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,6 +195,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&uempty[i], 1 + kFgEpiWarps);
     }
     mbar_init(mma_done, 1);
+    mbar_init(sched_ready, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -203,10 +213,20 @@ __global__ void __launch_bounds__(192, 1)
       mbar_expect_tx(&full[kc], C::kABytes);
       tma_load_4d_hint(tiles + kc * C::kStageBytes, mA, &full[kc], kc * kBK, mb0 * kBM, 0, ec, pol_w);
     }
-    const int kc1 = min(args.kc_gu, npre0 + args.pre_l2_chunks);
-    for (int kc = npre0; kc < kc1; ++kc) tma_prefetch_4d(mA, kc * kBK, mb0 * kBM, 0, ec);
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  const uint64_t limit = g_wait_timeout_ns;
+  // barriers and TMEM are published before the wait: no CTA-wide barrier follows it
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if (warp == 3 && lane == 0) {
+    // an epilogue warp, idle until the first unit's MMAs: descriptors, and
+    // further k-chunks of the first unit to L2, off the producer's path
     prefetch_tmap(&mGuR);
     prefetch_tmap(&mGuS);
     prefetch_tmap(&mDnR);
@@ -214,46 +234,113 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&mXr);
     prefetch_tmap(&mXs);
     prefetch_tmap(&mAct);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  }
-  griddep_wait();  // barriers, tensor maps and TMEM are set up; the grouping is read from here on
-  if (warp == 2) {
-    const int kT = args.offsets[args.E];
-    for (int e = lane; e < n_exp; e += 32) {
-      if (e < args.E) {
-        const int o0 = args.offsets[e], o1 = args.offsets[e + 1];
-        sch->xrow[e] = o0;
-        sch->arow[e] = o0;
-        sch->n[e] = o1 - o0;
-      } else {
-        const int s = e - args.E;
-        sch->xrow[e] = 0;
-        sch->arow[e] = kT + s * args.T;
-        sch->n[e] = args.T;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) {
-      int acc = 0;
-      for (int e = 0; e < n_exp; ++e) {
-        sch->pref[e] = acc;
-        const int nt = cdiv(sch->n[e], NMAX);
-        acc += args.static_first ? max(0, nt - 1) : nt;
-      }
-      sch->pref[n_exp] = acc;
+    if (npre0 > 0) {
+      const int e0 = blockIdx.x / args.mblk_gu, mb0 = blockIdx.x - e0 * args.mblk_gu;
+      const bool sh = e0 >= args.E;
+      const int kc1 = min(args.kc_gu, npre0 + args.pre_l2_chunks);
+      for (int kc = npre0; kc < kc1; ++kc) tma_prefetch_4d(sh ? &mGuS : &mGuR, kc * kBK, mb0 * kBM, 0, sh ? e0 - args.E : e0);
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  griddep_wait();  // the grouping is read from here on
 
-  const uint32_t tmem_base = *tmem_slot;
-  const int n_tiles = sch->pref[n_exp] + (args.static_first ? n_exp : 0);
-  const int total = n_tiles * (args.mblk_gu + args.mblk_dn);
-  const uint64_t limit = g_wait_timeout_ns;
+  // static_first: every role decodes the fixed first unit itself. The producer
+  // and the MMA issuer take it as a full tile whose token rows are known
+  // without the offsets (rows past the expert's tokens are computed and
+  // dropped), so its token rows are requested right after the wait; the
+  // epilogue reads the expert's row count and output rows from the offsets.
+  const bool epi = warp >= 2;
+  const int kT = epi ? args.offsets[args.E] : 0;  // routed rows; shared expert s owns rows kT + s T ..
+  [[maybe_unused]] const int rows_total = kT + args.S * args.T;  // bound of the epilogue's row checks
+  const int first_u = args.static_first ? (int)blockIdx.x : -1;
+  FgUnit first{};
+  if (args.static_first) {
+    const int e0 = blockIdx.x / args.mblk_gu;
+    first.tile = first.e = e0;
+    first.mb = blockIdx.x - e0 * args.mblk_gu;
+    const bool routed = e0 < args.E;
+    first.xrow = routed ? e0 * NMAX : 0;
+    first.nrows = NMAX;
+    first.arow = -1;
+    if (epi) {
+      int n;
+      if (routed) {
+        const int o0 = args.offsets[e0], o1 = args.offsets[e0 + 1];
+        first.arow = o0;
+        n = o1 - o0;
+      } else {
+        first.arow = kT + (e0 - args.E) * args.T;
+        n = args.T;
+      }
+      first.nrows = max(0, min(NMAX, n));
+    }
+  }
+  if (warp == 2) {
+    // the schedule: rows and tile prefix of every expert, kPer experts per lane
+    constexpr int kPer = (kMaxExperts + 31) / 32;
+    int o[kPer + 1];
+#pragma unroll
+    for (int i = 0; i <= kPer; ++i) {  // every offset this lane needs, requested at once
+      const int e = lane * kPer + i;
+      o[i] = e <= args.E ? args.offsets[e] : 0;
+    }
+    const int xbase = args.static_first ? args.E * NMAX : 0;  // further tiles' token rows
+    int cnt[kPer], local = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      int n = 0;
+      if (e < n_exp) {
+        const bool routed = e < args.E;
+        n = routed ? o[i + 1] - o[i] : args.T;
+        sch->xrow[e] = routed ? xbase + o[i] : 0;
+        sch->arow[e] = routed ? o[i] : kT + (e - args.E) * args.T;
+        sch->n[e] = n;
+      }
+      const int nt = cdiv(n, NMAX);
+      cnt[i] = e < n_exp ? (args.static_first ? max(0, nt - 1) : nt) : 0;
+      local += cnt[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    int run = incl - local;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      if (e < n_exp) sch->pref[e] = run;
+      run += cnt[i];
+    }
+    if (lane == 31) sch->pref[n_exp] = incl;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sched_ready);  // releases the schedule to the other roles
+  }
+  // every unit but the fixed first one is decoded from the schedule; each role
+  // waits for it once
+  bool sched_seen = false;
+  auto wait_sched = [&](int site) -> bool {
+    if (!sched_seen) {
+      if (!mbar_wait(sched_ready, 0, limit)) {
+        record_error(kErrTimeout, site);
+        *abort_flag = 1;
+        return false;
+      }
+      sched_seen = true;
+    }
+    return true;
+  };
+  auto decode = [&](int u, FgUnit& un, int site) -> bool {
+    if (u == first_u) {
+      un = first;
+      return true;
+    }
+    if (!wait_sched(site)) return false;
+    un = fg_decode(u, *sch, n_exp, args, NMAX);
+    return true;
+  };
+
   int32_t* ticket = args.sched;
   int32_t* ready = args.sched + 1;
   const int ready_target = args.mblk_gu * kFgEpiWarps;
@@ -278,15 +365,30 @@ __global__ void __launch_bounds__(192, 1)
       const int tbase = args.static_first ? (int)gridDim.x : 0;  // tickets after the fixed first units
       int next_u = args.static_first ? (int)blockIdx.x : atomicAdd(ticket, 1);
       bool pre_pending = npre0 > 0;  // stages 0 .. npre0-1 armed before the wait, not yet handed on
+      int total = -1;  // units of this launch, once the schedule is known
       while (true) {
         int u = next_u;
-        if (u >= total || *abort_flag) u = -1;
-        if (u >= 0) next_u = tbase + atomicAdd(ticket, 1);
+        if (u >= 0 && u != first_u) {
+          if (total < 0)
+            total = wait_sched(139) ? (sch->pref[n_exp] + (args.static_first ? n_exp : 0)) *
+                                          (args.mblk_gu + args.mblk_dn)
+                                    : 0;
+          if (u >= total) u = -1;
+        }
+        if (*abort_flag) u = -1;
         const bool pre_unit = pre_pending && u >= 0;  // the first unit: its weight stages are armed
+        // the fixed first unit asks for its successor only once its armed stages
+        // have their token rows requested: every CTA starts it at once, and the
+        // ticket's round trip is not on the way to the first MMA
+        bool want_ticket = u >= 0;
+        if (want_ticket && !pre_unit) {
+          next_u = tbase + atomicAdd(ticket, 1);
+          want_ticket = false;
+        }
         FgUnit un{};
         if (u >= 0) {
-          un = fg_decode(u, *sch, n_exp, args, NMAX);
-          if (un.nrows == 0 && !pre_unit) continue;  // a tile without tokens: nothing to compute
+          if (!decode(u, un, 139)) u = -1;
+          else if (un.nrows == 0 && !pre_unit) continue;  // a tile without tokens: nothing to compute
         }
         if (!mbar_wait(&uempty[slot], rphase ^ 1, limit)) {
           record_error(kErrTimeout, 130);
@@ -308,6 +410,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_arrive(&full[stage]);
             next_stage();
           }
+          if (want_ticket) next_u = tbase + atomicAdd(ticket, 1);
           continue;
         }
         const bool shared = un.e >= args.E;
@@ -346,6 +449,10 @@ __global__ void __launch_bounds__(192, 1)
               tma_load_4d_hint(st, mA, &full[stage], kc * kBK, arow, 0, ecoord, pol_w);
           }
           if (kc >= npre) load_b(stage, kc);
+          if (want_ticket && kc + 1 >= npre0) {
+            next_u = tbase + atomicAdd(ticket, 1);
+            want_ticket = false;
+          }
           if (kc + 1 == npre) {
             // every stage of the prefetch holds its weights in flight: now wait for the tile
             const uint64_t t0 = globaltimer();
@@ -393,7 +500,8 @@ __global__ void __launch_bounds__(192, 1)
           rphase ^= 1;
         }
         if (u < 0 || *abort_flag) break;
-        const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
+        FgUnit un;
+        if (!decode(u, un, 148)) break;
         if (un.nrows == 0) {  // the pre-armed unit of an unused expert: release its stages
           bool ok = true;
           for (int kc = 0; kc < npre0; ++kc) {
@@ -476,8 +584,9 @@ __global__ void __launch_bounds__(192, 1)
         rphase ^= 1;
       }
       if (u < 0 || *abort_flag) break;
-      const FgUnit un = fg_decode(u, *sch, n_exp, args, NMAX);
-      if (un.nrows == 0) continue;  // nothing was computed for it
+      FgUnit un;
+      if (!decode(u, un, 149)) break;
+      if (un.nrows == 0 && u != first_u) continue;  // nothing was computed for it
       const int ab = lu & 1;
       const uint32_t ap = (lu >> 1) & 1;
       ++lu;
@@ -488,8 +597,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       // the unit's rows lie inside the activation / output buffers: routed rows, then S x T shared rows
-      const bool rows_ok = VG_IN_BOUNDS(un.arow >= 0 && un.arow + un.nrows <= sch->arow[args.E] + args.S * args.T,
-                                        404);
+      const bool rows_ok = VG_IN_BOUNDS(un.arow >= 0 && un.arow + un.nrows <= rows_total, 404);
       const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + ab * C::kAccCols;
       if (un.down) {
         const int ld = args.mblk_dn * 2 * kBM;

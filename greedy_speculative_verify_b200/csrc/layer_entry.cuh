@@ -50,7 +50,12 @@ struct EntryArgs {
   int32_t* offsets;           // [65]
   int32_t* perm;              // [T k]
   int32_t* inv;               // [T k]
-  __nv_bfloat16* x_perm;      // [T k, H]
+  // x_perm rows: primary_rows == 0: permutation order, [T k, H]; otherwise the
+  // first primary_rows rows of expert e's segment at e * primary_rows and the
+  // rest at 64 primary_rows + (position in the permutation), so the first tile
+  // of every expert lies where the expert kernel can find it before the offsets
+  __nv_bfloat16* x_perm;
+  int32_t primary_rows;
   int32_t* counts;            // [grid, 64] per-CTA assignment counts (scratch)
   int32_t* sched;             // expert kernel's counters, cleared here
   int32_t sched_len;
@@ -79,6 +84,18 @@ constexpr int kEntryMaxGridDev = 160;                  // CTAs of the kernel at 
 // fp32, plus 1 KB alignment slack.
 __host__ __device__ constexpr int layer_entry_smem() {
   return 1024 + kRouterE * kEntryH * 2 + kEntryMaxOwn * kEntryH * 2 + kEntryPassTok * kEntryH * 4;
+}
+
+// L2 prefetch of n_prefetch weight blocks in 1 MB pieces, spread over the CTAs.
+__device__ __forceinline__ void entry_l2_prefetch(const EntryArgs& a, int c, int G) {
+  if (a.n_prefetch <= 0) return;
+  constexpr uint32_t kPiece = 1u << 20;
+  const uint32_t pieces_per = cdiv((int)a.prefetch_bytes, (int)kPiece);
+  for (uint32_t i = c; i < (uint32_t)a.n_prefetch * pieces_per; i += G) {
+    const uint32_t blk = i / pieces_per, pc = i - blk * pieces_per;
+    const uint32_t off = pc * kPiece;
+    bulk_prefetch_l2(a.prefetch_base + blk * a.prefetch_stride + off, min(kPiece, a.prefetch_bytes - off));
+  }
 }
 
 // NT quarter chains (one per token) over the thread's quarter of h; each
@@ -155,15 +172,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
       const int e = u / a.pf_mblk, mb = u - e * a.pf_mblk;
       for (int kc = 0; kc < a.pf_chunks; ++kc) tma_prefetch_4d(&mGu, kc * 64, mb * 128, 0, e);
     }
-    if (a.n_prefetch > 0) {
-      constexpr uint32_t kPiece = 1u << 20;
-      const uint32_t pieces_per = cdiv((int)a.prefetch_bytes, (int)kPiece);
-      for (uint32_t i = c; i < (uint32_t)a.n_prefetch * pieces_per; i += G) {
-        const uint32_t blk = i / pieces_per, pc = i - blk * pieces_per;
-        const uint32_t off = pc * kPiece;
-        bulk_prefetch_l2(a.prefetch_base + blk * a.prefetch_stride + off, min(kPiece, a.prefetch_bytes - off));
-      }
-    }
+    entry_l2_prefetch(a, c, G);  // the expert kernel's first weights, to L2 while this kernel routes
   }
   if (tid < kRouterE) cnt_s[tid] = 0;
   __syncthreads();
@@ -317,6 +326,9 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
     if (VG_IN_BOUNDS((unsigned)my_pos < (unsigned)N && a_begin + tid < N, 402)) {
       a.perm[my_pos] = a_begin + tid;
       a.inv[a_begin + tid] = my_pos;
+      const int r = pre_s[key] + rank;  // rank within the expert's segment
+      const int P = a.primary_rows;
+      my_pos = P == 0 ? my_pos : r < P ? key * P + r : kRouterE * P + my_pos;  // the row of x_perm
     } else {
       my_pos = -1;
     }
@@ -324,8 +336,9 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   __syncthreads();  // every rank was taken from idx_s before it is overwritten
   if (tid < n_own * K) idx_s[tid] = my_pos;
   __syncthreads();
+  [[maybe_unused]] const int xperm_rows = N + kRouterE * a.primary_rows;  // bound of the gather checks
   for (int i = warp; i < n_own * K; i += blockDim.x / 32) {
-    if (!VG_IN_BOUNDS((unsigned)idx_s[i] < (unsigned)N, 403)) continue;
+    if (!VG_IN_BOUNDS((unsigned)idx_s[i] < (unsigned)xperm_rows, 403)) continue;
     const uint4* src = reinterpret_cast<const uint4*>(xo + (size_t)(i / K) * H);
     uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (size_t)idx_s[i] * H);
     for (int cc = lane; cc < H / 8; cc += 32) dst[cc] = src[cc];

@@ -40,7 +40,7 @@ constexpr int kEntryMaxGrid = 256;  // CTAs of the layer-entry kernel at most
 #define VG_SMALL_ENTRY_PREFETCH_MB 0
 #endif
 #ifndef VG_PRE_L2_CHUNKS
-#define VG_PRE_L2_CHUNKS 15
+#define VG_PRE_L2_CHUNKS 0
 #endif
 #ifndef VG_ENTRY_PF_UNITS
 #define VG_ENTRY_PF_UNITS 0
@@ -209,7 +209,13 @@ struct MoeWs {
 // Tile width of the expert GEMMs: 16-token tiles (six pipeline stages) for a
 // handful of tokens, 64-token tiles (five stages) at decode sizes, 128-token
 // tiles for prefill-sized segments.
+static_assert(kTopK <= vg::kCombineMaxK && kS <= vg::kCombineMaxS, "the combine's unrolled loads cover k and S");
+
 int expert_tile(int T) { return T <= 16 ? 16 : T <= 1024 ? 64 : 128; }
+
+// Rows of x_perm beyond the T k assignments: with fixed first units (64-token
+// tiles) every routed expert's first tile has its own 64 rows ahead of them.
+size_t xperm_extra_rows(int T) { return expert_tile(T) == 64 ? (size_t)kE * 64 : 0; }
 
 // Upper bound of the expert GEMMs' token tiles: routed segments cut at the tile
 // width plus one partial tile per routed expert, plus the shared experts' tiles.
@@ -217,6 +223,12 @@ int max_tiles(int T) {
   const int nt = expert_tile(T);
   return vg::cdiv(T * kTopK, nt) + kE + kS * vg::cdiv(T, nt);
 }
+
+// CTAs of the expert kernel: one per SM, at most one per unit.
+int expert_grid(const DevState* dev, int T) {
+  return std::min(dev->sms, (kI / vg::kBM + kH / (2 * vg::kBM)) * max_tiles(T));
+}
+
 
 MoeWs moe_layout(int T) {
   const size_t N = (size_t)T * kTopK;
@@ -233,7 +245,7 @@ MoeWs moe_layout(int T) {
   L.offsets = take((kE + 1) * 4);
   L.perm = take(N * 4);
   L.inv = take(N * 4);
-  L.xperm = take(N * kH * 2);
+  L.xperm = take((N + xperm_extra_rows(T)) * kH * 2);
   L.act = take((size_t)(kTopK + kS) * T * kI * 2);
   L.o = take((size_t)(kTopK + kS) * T * kH * 2);
   L.ccnt = take(nch * kE * 4);
@@ -292,12 +304,17 @@ bool entry_small_path(const DevState* dev, int T) {
   return vg::cdiv(T, vg::kEsTok) <= std::min(dev->sms, vg::kEsMaxGrid);
 #endif
 }
+bool small_path(const DevState* dev, int T);
+int expert_grid(const DevState* dev, int T);
 bool static_first_units(const DevState* dev, int T) {
 #ifdef VG_NO_STATIC_FIRST
   return false;
 #endif
+  // the layer-entry kernel lays out the token rows of the fixed first tiles, and
+  // every CTA of the expert kernel has a primary gate/up unit of its own
   return T >= kStaticFirstMinT && vg::cdiv(T, vg::kEsTok) <= std::min(dev->sms, vg::kEsMaxGrid) &&
-         expert_tile(T) == 64;
+         expert_tile(T) == 64 && !entry_small_path(dev, T) && small_path(dev, T) &&
+         expert_grid(dev, T) <= (kE + kS) * (kI / vg::kBM);
 }
 
 // The layer-entry kernel takes decode sizes: at most kEntryMaxOwn tokens per CTA
@@ -378,6 +395,7 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     a.perm = b.perm;
     a.inv = b.inv;
     a.x_perm = b.xperm;
+    a.primary_rows = static_first_units(dev, T) ? 64 : 0;
     a.counts = b.ecnt;
     a.sched = b.sched;
     a.sched_len = b.sched_len;
@@ -462,7 +480,7 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   // down as (k, row, expert): one box = 256 rows, two M tiles
   const uint64_t dDn[3] = {kI, kH, kE}, dDnS[3] = {kI, kH, kS}, sDn[2] = {kI * 2, estride};
   const uint32_t bDn[3] = {kBK, 2 * kBM, 1};
-  const uint64_t dXr[2] = {kH, (uint64_t)N}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
+  const uint64_t dXr[2] = {kH, (uint64_t)(N + (static_first_units(dev, T) ? kE * 64 : 0))}, dXs[2] = {kH, (uint64_t)T}, sX[1] = {kH * 2};
   const uint64_t dAct[2] = {kI, (uint64_t)(kTopK + kS) * T}, sAct[1] = {kI * 2};
   const int nt = expert_tile(T);
   // token-major kernel (128-token tiles): its token operand is one 128-row box;
@@ -496,8 +514,8 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
   a.sched = b.sched;
   a.act = b.act;
   a.out = b.o;
-  const int grid = min(dev->sms, (a.mblk_gu + a.mblk_dn) * max_tiles(T));
-  a.static_first = static_first_units(dev, T) && grid <= (kE + kS) * a.mblk_gu ? 1 : 0;
+  const int grid = expert_grid(dev, T);
+  a.static_first = static_first_units(dev, T) ? 1 : 0;
   a.pre_l2_chunks = kPreL2Chunks;
   ProfScope ps(VG_KERNEL_EXPERTS, s);
   const cudaError_t e =

@@ -41,9 +41,10 @@ def test_workspace_queries(lib):
     d = vgv.MOE_DIMS
     w128 = vgv.vg_moe_workspace_bytes(d, 128)
     N = 128 * 6
-    # routing tables, permutation, gathered rows, activations, expert outputs;
-    # above that only small scratch (logits, per-CTA counts, scheduling counters)
-    floor = 4 * N * 4 + N * 1280 * 2 + 8 * 128 * 896 * 2 + 8 * 128 * 1280 * 2
+    # routing tables, permutation, gathered rows (at 64-token tiles also 64 rows
+    # for the first tile of each of the 64 routed experts), activations, expert
+    # outputs; above that only small scratch (logits, per-CTA counts, counters)
+    floor = 4 * N * 4 + (N + 64 * 64) * 1280 * 2 + 8 * 128 * 896 * 2 + 8 * 128 * 1280 * 2
     assert floor <= w128 < floor + 160 * 1024
     assert vgv.vg_moe_workspace_bytes(d, 256) > w128
     assert vgv.vg_moe_stack_workspace_bytes(d, 128) >= w128 + 2 * 128 * 1280 * 2
