@@ -101,33 +101,50 @@ __device__ __forceinline__ void entry_l2_prefetch(const EntryArgs& a, int c, int
 // NT quarter chains (one per token) over the thread's quarter of h; each
 // weight pair is unpacked once for all NT tokens. `wq` is the thread's row in
 // the swizzled tile of its quarter's first 64 columns, `xq` the quarter's
-// first fp32 input of token 0 (token j at + j * kEntryH).
+// first fp32 input of token 0 (token j at + j * kEntryH). The chains run in
+// 40 steps of 8 columns; the next step's weights and inputs are loaded while
+// the current step's 8 FMAs run.
 template <int NT>
 __device__ __forceinline__ void quarter_chains(const uint8_t* wq, int sw, const float* xq, float* acc) {
-  constexpr int kTiles = kEntryH / 4 / 64;  // a quarter spans 5 tiles of 64 columns
+  constexpr int kSteps = kEntryH / 4 / 8;  // 40 steps of 8 columns
 #pragma unroll
   for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
-#pragma unroll 1
-  for (int m = 0; m < kTiles; ++m) {
+  auto wptr = [&](int i) {
+    return reinterpret_cast<const uint4*>(wq + (i >> 3) * 8192 + (((i & 7) ^ sw) << 4));
+  };
+  uint4 wv = *wptr(0);
+  float4 xa[NT], xb[NT];
 #pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8) {  // 16-byte slot q8 of the row: columns 8 q8 .. 8 q8 + 7
-      const uint4 wv = *reinterpret_cast<const uint4*>(wq + m * 8192 + ((q8 ^ sw) << 4));
-      const float w[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
-                          bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
+  for (int j = 0; j < NT; ++j) {
+    xa[j] = reinterpret_cast<const float4*>(xq + j * kEntryH)[0];
+    xb[j] = reinterpret_cast<const float4*>(xq + j * kEntryH)[1];
+  }
+#pragma unroll 4
+  for (int i = 0; i < kSteps; ++i) {
+    const int in = i + 1 < kSteps ? i + 1 : i;  // the last step reloads its own data
+    const uint4 wn = *wptr(in);
+    float4 xan[NT], xbn[NT];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const float4* xv = reinterpret_cast<const float4*>(xq + j * kEntryH + m * 64 + q8 * 8);
-        const float4 x0 = xv[0], x1 = xv[1];
-        acc[j] = __fmaf_rn(x0.x, w[0], acc[j]);
-        acc[j] = __fmaf_rn(x0.y, w[1], acc[j]);
-        acc[j] = __fmaf_rn(x0.z, w[2], acc[j]);
-        acc[j] = __fmaf_rn(x0.w, w[3], acc[j]);
-        acc[j] = __fmaf_rn(x1.x, w[4], acc[j]);
-        acc[j] = __fmaf_rn(x1.y, w[5], acc[j]);
-        acc[j] = __fmaf_rn(x1.z, w[6], acc[j]);
-        acc[j] = __fmaf_rn(x1.w, w[7], acc[j]);
-      }
+    for (int j = 0; j < NT; ++j) {
+      xan[j] = reinterpret_cast<const float4*>(xq + j * kEntryH + in * 8)[0];
+      xbn[j] = reinterpret_cast<const float4*>(xq + j * kEntryH + in * 8)[1];
     }
+    const float w[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
+                        bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      acc[j] = __fmaf_rn(xa[j].x, w[0], acc[j]);
+      acc[j] = __fmaf_rn(xa[j].y, w[1], acc[j]);
+      acc[j] = __fmaf_rn(xa[j].z, w[2], acc[j]);
+      acc[j] = __fmaf_rn(xa[j].w, w[3], acc[j]);
+      acc[j] = __fmaf_rn(xb[j].x, w[4], acc[j]);
+      acc[j] = __fmaf_rn(xb[j].y, w[5], acc[j]);
+      acc[j] = __fmaf_rn(xb[j].z, w[6], acc[j]);
+      acc[j] = __fmaf_rn(xb[j].w, w[7], acc[j]);
+      xa[j] = xan[j];
+      xb[j] = xbn[j];
+    }
+    wv = wn;
   }
 }
 
