@@ -55,8 +55,8 @@ NOMINAL_HBM_GBS = 8000.0        # "about 8 TB/s", the nominal figure the decode 
 # DRAM bytes (read + write) of one expert-GEMM launch at 128 tokens from one ncu
 # capture, with the SHA-256 (first 16 hex digits) of the kernel source it was
 # taken on; the bench reports it only while the source is unchanged.
-EXPERT_TRAFFIC = {"bytes": 462.35e6, "source": "greedy_speculative_verify_b200/csrc/gemm_moe.cuh",
-                  "source_sha16": "421d678ef8d4d9bb", "profile": "profiles/moe_expert_gemms_t128.md"}
+EXPERT_TRAFFIC = {"bytes": 465.68e6, "source": "greedy_speculative_verify_b200/csrc/gemm_moe.cuh",
+                  "source_sha16": "75dda351e238651c", "profile": "profiles/moe_expert_gemms_t128.md"}
 
 
 def _traffic(rec):

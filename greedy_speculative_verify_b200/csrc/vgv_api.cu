@@ -157,7 +157,8 @@ vg_status device_state(DevState** out) {
           cudaFuncSetAttribute(vg::moe_expert_gemms<64>, kC, kMax) != cudaSuccess ||
           cudaFuncSetAttribute(vg::moe_expert_gemms<128>, kC, kMax) != cudaSuccess ||
           cudaFuncSetAttribute(vg::moe_expert_gemms_tm, kC, kMax) != cudaSuccess ||
-          cudaFuncSetAttribute(vg::moe_combine, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_combine<true>, kC, kMax) != cudaSuccess ||
+          cudaFuncSetAttribute(vg::moe_combine<false>, kC, kMax) != cudaSuccess ||
           cudaFuncSetAttribute(vg::lmhead_argmax_accept, kC, kMax) != cudaSuccess ||
           cudaFuncSetAttribute(vg::embed_rows, kC, kMax) != cudaSuccess ||
           cudaFuncSetAttribute(vg::spec_rows, kC, kMax) != cudaSuccess ||
@@ -209,6 +210,7 @@ struct MoeWs {
 // Tile width of the expert GEMMs: 16-token tiles (six pipeline stages) for a
 // handful of tokens, 64-token tiles (five stages) at decode sizes, 128-token
 // tiles for prefill-sized segments.
+constexpr int kCombineAllLoadsMaxT = 1024;  // tokens up to which the combine issues all loads first
 static_assert(kTopK <= vg::kCombineMaxK && kS <= vg::kCombineMaxS, "the combine's unrolled loads cover k and S");
 
 int expert_tile(int T) { return T <= 16 ? 16 : T <= 1024 ? 64 : 128; }
@@ -443,8 +445,8 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
   }
   const __nv_bfloat16* xcur = x_in;
   if (prev) {
-    moe_combine<<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(prev->x, prev->b->o, prev->b->inv, prev->b->gw, T, kH,
-                                                       kTopK, kS, 1, x_out);
+    moe_combine<false><<<cdiv(T * (kH / 8), 256), 256, 0, s>>>(prev->x, prev->b->o, prev->b->inv, prev->b->gw, T,
+                                                              kH, kTopK, kS, 1, x_out);
     xcur = x_out;
   }
   {
@@ -535,7 +537,9 @@ vg_status launch_experts(DevState* dev, int T, const void* x, const void* expert
 vg_status launch_combine(int T, const void* x, const LayerBufs& b, int add_residual, void* out, cudaStream_t s) {
   using namespace vg;
   ProfScope ps(VG_KERNEL_COMBINE, s);
-  const cudaError_t e = launch_dep(moe_combine, cdiv(T * (kH / 8), 256), 256, 0, s, Launch::kPlain,
+  // few tokens: every load of a thread at once (latency); many: one row at a time (throughput)
+  const cudaError_t e = launch_dep(T <= kCombineAllLoadsMaxT ? moe_combine<true> : moe_combine<false>,
+                                   cdiv(T * (kH / 8), 256), 256, 0, s, Launch::kPlain,
                                    static_cast<const __nv_bfloat16*>(x), (const __nv_bfloat16*)b.o,
                                    (const int32_t*)b.inv, (const float*)b.gw, T, kH, kTopK, kS, add_residual,
                                    static_cast<__nv_bfloat16*>(out));
