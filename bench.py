@@ -716,6 +716,30 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def measure_box_copy(dev, nbytes=2 << 30):
+    """This GPU's device-to-device copy rate now (read + write bytes of a 2 GiB
+    copy, best of 5): context for the spread between boxes of the pool. The
+    roofline's peak stays the measured peak of MEASURED_PEAKS.json."""
+    import torch
+
+    src = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    src.fill_(1)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = float("inf")
+    for _ in range(5):
+        torch.cuda.synchronize()
+        e0.record()
+        dst.copy_(src)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del src, dst
+    torch.cuda.empty_cache()
+    return {"gbs": 2 * nbytes / (best / 1e3) / 1e9, "bytes_copied": nbytes,
+            "rule": "read + write bytes of one 2 GiB device-to-device copy (torch), best of 5, after the step"}
+
+
 def run_gpu(args, rank, world, local):
     import torch
     import torch.distributed as dist
@@ -908,6 +932,7 @@ def run_gpu(args, rank, world, local):
 
     peak, peak_kind = _peaks()
     step_bytes = step_weight_bytes(n_touched)
+    box_copy = measure_box_copy(dev)
     line = {
         "metric": METRIC, "value": tokens_all / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -931,8 +956,10 @@ def run_gpu(args, rank, world, local):
                           "frac_of_measured": step_bytes / (ms / 1e3) / 1e9 / peak,
                           "frac_of_nominal_8tbs": step_bytes / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS,
                           "measured_peak_gbs": peak, "peak_source": f"{peak_kind} hbm_gbs",
+                          "frac_of_this_box_copy": step_bytes / (ms / 1e3) / 1e9 / box_copy["gbs"],
                           "bytes_rule": "sum over layers of router + (touched + 2 shared) experts' weights, "
                                         "+ the LM head; activations excluded"},
+        "box_copy": box_copy,
         "breakdown_ms_per_step": breakdown,
         "clocks": clk,
         "cpu_baseline": cpu,
