@@ -98,23 +98,38 @@ __global__ void __launch_bounds__(1024) expert_hist_chunks(const int32_t* __rest
 }
 
 // Pass 2 (one block of 64 threads): offsets and each chunk's per-expert base.
-__global__ void __launch_bounds__(64) expert_scan_chunks(const int32_t* __restrict__ chunk_cnt, int nchunks, int N,
-                                                         int32_t* __restrict__ offsets,
-                                                         int32_t* __restrict__ chunk_base,
-                                                         int32_t* __restrict__ sched, int sched_len) {
+__global__ void __launch_bounds__(1024) expert_scan_chunks(const int32_t* __restrict__ chunk_cnt, int nchunks, int N,
+                                                           int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ chunk_base,
+                                                           int32_t* __restrict__ sched, int sched_len) {
+  // thread (slice sl, expert e) sums the counts of a contiguous range of
+  // chunks, requested together; the slices' sums give each expert's total and
+  // each range's starting point (integer sums: the order does not matter)
+  constexpr int kSl = 1024 / kSortE;
+  __shared__ int part[kSl][kSortE];
   __shared__ int tot[kSortE], off[kSortE];
-  const int e = threadIdx.x;
-  for (int i = e; i < sched_len; i += blockDim.x) sched[i] = 0;  // expert GEMM tickets + readiness
+  const int e = threadIdx.x % kSortE, sl = threadIdx.x / kSortE;
+  for (int i = threadIdx.x; i < sched_len; i += blockDim.x) sched[i] = 0;  // expert GEMM tickets + readiness
+  const int R = (nchunks + kSl - 1) / kSl, c0 = min(nchunks, sl * R), c1 = min(nchunks, c0 + R);
   int s = 0;
-  for (int c = 0; c < nchunks; ++c) s += chunk_cnt[c * kSortE + e];
-  tot[e] = s;
+#pragma unroll 8
+  for (int c = c0; c < c1; ++c) s += chunk_cnt[c * kSortE + e];
+  part[sl][e] = s;
   __syncthreads();
-  if (e < 32) scan64_warp(tot, off, e);
+  if (threadIdx.x < kSortE) {
+    int t = 0;
+    for (int j = 0; j < kSl; ++j) t += part[j][e];
+    tot[e] = t;
+  }
   __syncthreads();
-  offsets[e] = off[e];
-  if (e == 0) offsets[kSortE] = N;
+  if (threadIdx.x < 32) scan64_warp(tot, off, threadIdx.x);
+  __syncthreads();
+  if (threadIdx.x < kSortE) offsets[e] = off[e];
+  if (threadIdx.x == 0) offsets[kSortE] = N;
   int run = off[e];
-  for (int c = 0; c < nchunks; ++c) {
+  for (int j = 0; j < sl; ++j) run += part[j][e];
+#pragma unroll 8
+  for (int c = c0; c < c1; ++c) {
     chunk_base[c * kSortE + e] = run;
     run += chunk_cnt[c * kSortE + e];
   }
@@ -143,9 +158,32 @@ __global__ void __launch_bounds__(1024) expert_scatter_chunks(const int32_t* __r
     inv[a] = pos;
   }
   __syncthreads();
-  for (int i = warp; i < kSortChunk; i += 32) {
-    const int p = pos_s[i];
-    if (p >= 0) gather_rows(x, x_perm, H, p, (base + i) / k);
+  if (H == 1280) {
+    // two rows per warp at a time, every 16-byte load of both issued before the stores
+    constexpr int kPer = 1280 / 8 / 32;  // 16-byte pieces per lane and row
+    const int lane = tid & 31;
+    for (int i = warp; i < kSortChunk; i += 64) {
+      const int i1 = i + 32;
+      const int p0 = pos_s[i], p1 = i1 < kSortChunk ? pos_s[i1] : -1;
+      uint4 v0[kPer], v1[kPer];
+      const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)((base + i) / k) * H);
+      const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)((base + i1) / k) * H);
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        if (p0 >= 0) v0[j] = __ldg(s0 + lane + 32 * j);
+        if (p1 >= 0) v1[j] = __ldg(s1 + lane + 32 * j);
+      }
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        if (p0 >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)p0 * H)[lane + 32 * j] = v0[j];
+        if (p1 >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)p1 * H)[lane + 32 * j] = v1[j];
+      }
+    }
+  } else {
+    for (int i = warp; i < kSortChunk; i += 32) {
+      const int p = pos_s[i];
+      if (p >= 0) gather_rows(x, x_perm, H, p, (base + i) / k);
+    }
   }
 }
 

@@ -459,7 +459,7 @@ vg_status launch_entry(DevState* dev, int T, const PrevCombine* prev, const __nv
     ProfScope ps(VG_KERNEL_GROUPING, s);
     const int nch = cdiv(N, kSortChunk);
     expert_hist_chunks<<<nch, 1024, 0, s>>>(b.idx, N, b.ccnt);
-    expert_scan_chunks<<<1, 64, 0, s>>>(b.ccnt, nch, N, b.offsets, b.cbase, b.sched, b.sched_len);
+    expert_scan_chunks<<<1, 1024, 0, s>>>(b.ccnt, nch, N, b.offsets, b.cbase, b.sched, b.sched_len);
     expert_scatter_chunks<<<nch, 1024, 0, s>>>(b.idx, N, kTopK, b.cbase, b.perm, b.inv, xcur, kH, b.xperm);
   }
   if (cudaGetLastError() != cudaSuccess) return VG_ERR_CUDA;
