@@ -204,6 +204,11 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
       const uint4 v = combine8(a.prev_x, a.prev_o, a.prev_inv, a.prev_gate, a.T, H, a.k, a.S, a.prev_add_residual, t, cc);
       reinterpret_cast<uint4*>(a.x_out + (size_t)t * H)[cc] = v;
       reinterpret_cast<uint4*>(xo + (size_t)tl * H)[cc] = v;
+      if (tl < kEntryPassTok) {  // the first pass's rows in fp32 too
+        float4* xf4 = reinterpret_cast<float4*>(xf + (size_t)tl * H + cc * 8);
+        xf4[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+        xf4[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+      }
     }
   } else if (n_own > 0) {
     if (tid == 0) {
@@ -225,11 +230,13 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   const int grp = tid >> 8, qq = (tid >> 6) & 3, e = tid & 63;
   for (int g0 = 0; ok && g0 < n_own; g0 += kEntryPassTok) {
     const int n_pass = min(kEntryPassTok, n_own - g0);
-    for (int i = tid; i < n_pass * H / 2; i += blockDim.x) {  // the pass's rows to fp32
-      const uint32_t v = reinterpret_cast<const uint32_t*>(xo + (size_t)g0 * H)[i];
-      reinterpret_cast<float2*>(xf)[i] = make_float2(bf16_lo(v), bf16_hi(v));
+    if (g0 > 0 || a.prev_o == nullptr) {  // the combine wrote the first pass's fp32 rows
+      for (int i = tid; i < n_pass * H / 2; i += blockDim.x) {  // the pass's rows to fp32
+        const uint32_t v = reinterpret_cast<const uint32_t*>(xo + (size_t)g0 * H)[i];
+        reinterpret_cast<float2*>(xf)[i] = make_float2(bf16_lo(v), bf16_hi(v));
+      }
+      __syncthreads();
     }
-    __syncthreads();
     const int tok0 = grp * kEntryGroupTok, n_grp = min(kEntryGroupTok, n_pass - tok0);  // warp-uniform
     if (n_grp > 0) {
       const uint8_t* wq = ws + qq * (HQ / 64) * 8192 + e * 128;
