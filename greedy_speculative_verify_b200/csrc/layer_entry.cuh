@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
   __shared__ __align__(8) uint64_t bars[2];                                       // weights, token rows
   __shared__ __align__(16) float part[4][kEntryPassTok][kRouterE];                // [quarter][token][expert]
   __shared__ float logit[kEntryPassTok][kRouterE];
-  __shared__ float mx_s[kEntryPassTok], sum_s[kEntryPassTok][2];
+  __shared__ float sum_s[kEntryPassTok][2];
   __shared__ int32_t idx_s[kEntryMaxOwn * K];
   __shared__ int cnt_s[kRouterE], tot_s[kRouterE], pre_s[kRouterE], off_s[kRouterE];
 
@@ -260,19 +260,19 @@ __global__ void __launch_bounds__(kEntryThreads, 1) moe_layer_entry(const __grid
       logit[tk][e] = l;
     }
     __syncthreads();
+    float mx = l;  // the token's largest logit, taken in the same scan
     if (tk < n_pass) {
       rank = 0;
 #pragma unroll 8
       for (int j = 0; j < kRouterE; ++j) {
         const float o = logit[tk][j];
         rank += (o > l || (o == l && j < e)) ? 1 : 0;
+        mx = fmaxf(mx, o);
       }
-      if (rank == 0) mx_s[tk] = l;
     }
-    __syncthreads();
     float ex = 0.0f;
     if (tk < n_pass) {
-      ex = expf(l - mx_s[tk]);
+      ex = expf(l - mx);
       float s = ex;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
