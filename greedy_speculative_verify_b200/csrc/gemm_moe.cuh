@@ -635,9 +635,8 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) {
         mbar_arrive(&tempty[ab]);
         if (!un.down) {
-          // release: the warp's activation rows (ordered before by __syncwarp)
-          // precede the count the down units acquire
-          asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ready + un.tile) : "memory");
+          __threadfence();
+          atomicAdd(ready + un.tile, 1);
         }
       }
     }
